@@ -1,0 +1,212 @@
+"""Pins of the CPU oracle against what the NOSA pages and the mathematics fix.
+
+Each test is chosen so that a plausible slip (a dropped bias, a wrong pooling
+order, a wrong index, a transposed operand, a wrong tie rule) fails it.
+The expected values come from closed forms, constructions whose answer is
+known by design, or special cases that reduce to textbook softmax attention.
+"""
+import numpy as np
+import pytest
+
+from oracle import OracleUnit
+from tests import cases
+
+FIXTURES = ["maxpool_two_stage.json", "gqa_group_sum.json", "tie_lower_index.json", "evict_two_stage.json"]
+
+
+@pytest.mark.parametrize("name", FIXTURES)
+def test_golden_selection(name):
+    spec = cases.load_fixture(name)
+    K, V, e, q = cases.build_fixture(spec)
+    u = OracleUnit(D=spec["D"], G=spec["G"], block=spec["block"], sub=spec["sub"], k_q=spec["k_q"],
+                   k_e=spec["k_e"], cap=64 * 64)
+    u.prefill(K, V, e)
+    z = np.zeros(spec["D"], np.uint16)
+    r = u.step(z, z, 0.0, q)
+    assert r["gq"].tolist() == spec["expect_gq"]
+    if "expect_ge" in spec:
+        assert r["ge"].tolist() == spec["expect_ge"]
+    assert r["sel"].tolist() == spec["expect_sel"]
+
+
+def test_tie_two_way_order():
+    spec = cases.load_fixture("tie_lower_index.json")
+    spec["k_q"] = 2
+    K, V, e, q = cases.build_fixture(spec)
+    u = OracleUnit(G=1, k_q=2, k_e=0, cap=4096)
+    u.prefill(K, V, e)
+    z = np.zeros(128, np.uint16)
+    assert u.step(z, z, 0.0, q)["gq"].tolist() == [1, 3]
+
+
+def test_compressed_keys_closed_form():
+    """Ramp keys: K[j][d] = (j mod 16)/16 * (+1 even d, -1 odd d) + (sub-block index mod 8)/2.
+    The mean over an aligned 16-token sub-block s is +-7.5/16 + (s mod 8)/2 exactly."""
+    L, D = 16 * 13 + 5, 128
+    j = np.arange(L)
+    sign = np.where(np.arange(D) % 2 == 0, 1.0, -1.0)
+    K = ((j % 16) / 16.0)[:, None] * sign[None, :] + (((j // 16) % 8) / 2.0)[:, None]
+    Kb = cases.f32_to_bf16_bits_exact(K.astype(np.float32))
+    u = OracleUnit(k_q=1, k_e=1, cap=4096)
+    u.prefill(Kb, Kb, np.zeros(L, np.float32))
+    ck = u.ck()
+    assert ck.shape == (13, D)
+    s = np.arange(13)
+    want = 7.5 / 16 * sign[None, :] + ((s % 8) / 2.0)[:, None]
+    assert np.array_equal(ck, want)
+
+
+def test_block_eviction_closed_form():
+    """One spike x > 0 in block 1 -> E_1 = x/16; a negative spike in block 2 leaves its max at 0."""
+    L = 64 * 4 + 3
+    e = np.zeros(L, np.float32)
+    e[64 + 37] = 3.0
+    e[128 + 5] = -7.0
+    z = np.zeros((L, 128), np.uint16)
+    u = OracleUnit(k_q=1, k_e=1, cap=4096)
+    u.prefill(z, z, e)
+    assert u.E().tolist() == [0.0, 3.0 / 16, 0.0, 0.0]
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_all_blocks_selected_equals_dense_softmax(G):
+    """With k_q >= number of candidates every block is selected, so the sparse
+    step must equal textbook softmax(q K^T / sqrt(D) + e) V over all L tokens."""
+    L0 = 699  # 10 complete blocks + a 59-token local block; the step adds one
+    K, V, e = cases.synthetic_unit(7, 0, 0, 1, L0 + 1)
+    q = cases.synthetic_queries(7, 0, 0, 1, G, 1)[0]
+    u = OracleUnit(G=G, k_q=16, k_e=4, cap=2048)
+    u.prefill(K[:L0], V[:L0], e[:L0])
+    r = u.step(K[L0], V[L0], float(e[L0]), q)
+    assert r["sel"].tolist() == list(range(11))
+    want = cases.textbook_attention(q, K, V, e, np.arange(L0 + 1), 1 / np.sqrt(128))
+    np.testing.assert_allclose(r["o"], want, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(u.dense(q), want, rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("G", [1, 8])
+def test_sparse_step_is_softmax_over_selected_tokens(G):
+    L0 = 64 * 45 + 17
+    K, V, e = cases.synthetic_unit(11, 2, 1, 0, L0 + 1)
+    q = cases.synthetic_queries(11, 2, 1, 0, G, 1)[0]
+    u = OracleUnit(G=G, k_q=4, k_e=6, cap=4096)
+    u.prefill(K[:L0], V[:L0], e[:L0])
+    r = u.step(K[L0], V[L0], float(e[L0]), q)
+    sel = r["sel"]
+    assert sel[-1] == L0 // 64 and len(sel) <= 4 + 6 + 1
+    assert sel[:-1].tolist() == sorted(set(r["gq"].tolist()) | set(r["ge"].tolist()))
+    tok = np.concatenate([np.arange(b * 64, min(b * 64 + 64, L0 + 1)) for b in sel])
+    want = cases.textbook_attention(q, K, V, e, tok, 1 / np.sqrt(128))
+    np.testing.assert_allclose(r["o"], want, rtol=1e-12, atol=1e-15)
+
+
+def _beats(sa, ia, sb, ib):
+    return sa > sb or (sa == sb and ia < ib)
+
+
+def test_topk_is_the_k_best_by_pairwise_check():
+    """Brute force: every selected block beats every unselected candidate."""
+    L0 = 64 * 60 + 3
+    K, V, e = cases.synthetic_unit(3, 0, 0, 0, L0 + 1)
+    q = cases.synthetic_queries(3, 0, 0, 0, 2, 1)[0]
+    u = OracleUnit(G=2, k_q=7, k_e=9, cap=8192)
+    u.prefill(K[:L0], V[:L0], e[:L0])
+    r = u.step(K[L0], V[L0], float(e[L0]), q)
+    s, E = r["scores"], u.E()
+    nb = r["nb_c"]
+    for chosen, score in ((r["gq"], s), (r["ge"], E[:nb])):
+        rest = sorted(set(range(nb)) - set(chosen.tolist()))
+        for a in chosen:
+            for b in rest:
+                assert _beats(score[a], a, score[b], b)
+    # Gamma_q comes out in rank order
+    for a, b in zip(r["gq"][:-1], r["gq"][1:]):
+        assert _beats(s[a], a, s[b], b)
+
+
+def test_locality_bound_is_tight_with_alternating_queries():
+    """Gamma_e = blocks 0..5 (highest eviction scores); the query alternates
+    between two orthogonal directions that each pick a different pair of
+    blocks, so Sel(t) shares exactly the 6 Gamma_e blocks with S(t-1):
+    gamma(t) = 6/8 = k_e/k, and exactly the 2 new Gamma_q blocks are fetched."""
+    nb, D = 100, 128
+    L0 = nb * 64 + 1
+    K = np.zeros((L0, D), np.float32)
+    for b in (10, 11):
+        K[b * 64:(b + 1) * 64, 0] = 1.0
+    for b in (20, 21):
+        K[b * 64:(b + 1) * 64, 1] = 1.0
+    e = np.zeros(L0, np.float32)
+    for b, val in zip(range(6), [5.0, 4.0, 3.0, 2.0, 1.5, 1.0]):
+        e[b * 64:(b + 1) * 64] = val
+    Kb = cases.f32_to_bf16_bits_exact(K)
+    u = OracleUnit(G=1, k_q=2, k_e=6, cap=8192)
+    u.prefill(Kb, Kb, e)
+    qa = np.zeros((1, D), np.float32); qa[0, 0] = 1.0
+    qb = np.zeros((1, D), np.float32); qb[0, 1] = 1.0
+    z = np.zeros(D, np.uint16)
+    for t in range(12):
+        q = cases.f32_to_bf16_bits_exact(qa if t % 2 == 0 else qb)
+        r = u.step(z, z, 0.0, q)
+        assert r["ge"].tolist() == [0, 1, 2, 3, 4, 5]
+        assert r["gq"].tolist() == ([10, 11] if t % 2 == 0 else [20, 21])
+        if t == 0:
+            assert r["n_fetch"] == 8  # cold cache: only the local block is resident after prefill
+        else:
+            assert r["n_overlap"] == 6 and r["gamma"] == 0.75 and r["n_fetch"] == 2
+    assert u.violations()["gamma"] == 0
+
+
+def test_incremental_eviction_sequence():
+    """Blocks complete during decode with eviction scores 1, 3, 2 (prefill),
+    then 2.5, 5, 0.5. With k_e = 2: {1,2} -> {1,3} -> {1,4} -> {1,4}; dropped
+    blocks never return."""
+    D = 128
+    Es = [1.0, 3.0, 2.0, 2.5, 5.0, 0.5]
+    L_all = 64 * len(Es) + 64
+    e = np.zeros(L_all, np.float32)
+    for b, val in enumerate(Es):
+        e[b * 64:(b + 1) * 64] = val
+    z = np.zeros((L_all, D), np.uint16)
+    u = OracleUnit(G=1, k_q=0, k_e=2, cap=4096)
+    L0 = 3 * 64 + 1
+    u.prefill(z[:L0], z[:L0], e[:L0])
+    q = np.zeros((1, D), np.uint16)
+    expect = {3: [1, 2], 4: [1, 3], 5: [1, 4], 6: [1, 4]}
+    seen = {}
+    for p in range(L0, 64 * 6 + 1):
+        r = u.step(z[p], z[p], float(e[p]), q)
+        seen[r["nb_c"]] = r["ge"].tolist()
+    assert seen == expect
+    v = u.violations()
+    assert v["reselect"] == 0 and v["incremental"] == 0
+
+
+@pytest.mark.parametrize("G,k_q,k_e", [(1, 4, 12), (8, 16, 48)])
+def test_invariants_over_many_steps(G, k_q, k_e):
+    """Random drifting queries over 150 steps that cross block boundaries:
+    gamma(t) >= k_e/k, no re-selection, incremental == brute-force Gamma_e,
+    fetches only from fresh Gamma_q blocks."""
+    L0, steps = 64 * 70 + 40, 150
+    K, V, e = cases.synthetic_unit(5, 1, 0, 1, L0 + steps)
+    qs = cases.synthetic_queries(5, 1, 0, 1, G, steps)
+    u = OracleUnit(G=G, k_q=k_q, k_e=k_e, cap=8192)
+    u.prefill(K[:L0], V[:L0], e[:L0])
+    for t in range(steps):
+        p = L0 + t
+        r = u.step(K[p], V[p], float(e[p]), qs[t])
+        if t >= 1:
+            assert r["gamma"] >= k_e / (k_q + k_e)
+            assert r["n_fetch"] <= k_q
+    v = u.violations()
+    assert v == {"gamma": 0, "reselect": 0, "incremental": 0, "fetch": 0, "steps": steps}
+
+
+def test_first_token_and_tiny_context():
+    """L = 1 after the append: no candidates, the output is the single value row."""
+    K, V, e = cases.synthetic_unit(1, 0, 0, 0, 1)
+    q = cases.synthetic_queries(1, 0, 0, 0, 2, 1)[0]
+    u = OracleUnit(G=2, k_q=4, k_e=4, cap=128)
+    r = u.step(K[0], V[0], float(e[0]), q)
+    assert r["sel"].tolist() == [0] and r["nb_c"] == 0
+    np.testing.assert_array_equal(r["o"], np.repeat(cases.bf16_bits_to_f64(V[0])[None], 2, 0))
