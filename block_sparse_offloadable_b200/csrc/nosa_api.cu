@@ -1,0 +1,388 @@
+// nosa_api.cu -- the C ABI of libnosa: argument validation, buffer sizes,
+// tensor maps and kernel launches.  Declarations and contracts: include/nosa.h.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <string.h>
+
+#include "nosa_internal.cuh"
+
+using namespace nosa;
+
+namespace {
+
+constexpr int64_t kMaxCtx = 1ll << 20;
+
+struct Geo {
+    int64_t units, nblk, nsub, nslots, max_sel, G;
+};
+
+bool geo_of(const nosa_config *c, Geo *g) {
+    if (nosa_validate_config(c) != NOSA_OK) return false;
+    g->units = (int64_t)c->batch * c->heads_kv;
+    g->nblk = c->max_ctx / kBlock;
+    g->nsub = c->max_ctx / kSub;
+    g->nslots = c->k_q + c->k_e + 2;
+    g->max_sel = c->k_q + c->k_e + 1;
+    g->G = c->heads_q / c->heads_kv;
+    return true;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Kind of memory behind p: cudaMemoryTypeDevice / Host / Managed / Unregistered.
+int mem_kind(const void *p, void **dev_addr) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return cudaMemoryTypeUnregistered;
+    }
+    if (dev_addr) *dev_addr = a.devicePointer;
+    return a.type;
+}
+
+bool is_device(const void *p) {
+    const int k = mem_kind(p, nullptr);
+    return k == cudaMemoryTypeDevice || k == cudaMemoryTypeManaged;
+}
+
+int check_dev(const void *p, bool need16) {
+    if (!p) return NOSA_ERR_PTR;
+    if (need16 && !aligned16(p)) return NOSA_ERR_PTR;
+    return is_device(p) ? NOSA_OK : NOSA_ERR_PTR;
+}
+
+// Device address of the KV store: device memory (offload 0) or mapped host memory (offload 1).
+int store_addr(const nosa_config *c, const nosa_state *st, uint8_t **out) {
+    if (!st->kv_store || !aligned16(st->kv_store)) return NOSA_ERR_PTR;
+    void *dev = nullptr;
+    const int k = mem_kind(st->kv_store, &dev);
+    if (c->offload) {
+        if (k != cudaMemoryTypeHost || !dev || !aligned16(dev)) return NOSA_ERR_PTR;
+    } else {
+        if (k != cudaMemoryTypeDevice && k != cudaMemoryTypeManaged) return NOSA_ERR_PTR;
+        dev = st->kv_store;
+    }
+    *out = static_cast<uint8_t *>(dev);
+    return NOSA_OK;
+}
+
+int check_state(const nosa_config *c, const nosa_state *st) {
+    if (!st) return NOSA_ERR_ARG;
+    int rc;
+    if ((rc = check_dev(st->evict_logit, true)) || (rc = check_dev(st->ck, true)) ||
+        (rc = check_dev(st->blk_evict, true)) || (rc = check_dev(st->gamma_n, false)) ||
+        (rc = check_dev(st->seq_len, false)) || (rc = check_dev(st->err, false)))
+        return rc;
+    if (c->k_e > 0 && (rc = check_dev(st->gamma_e, false))) return rc;
+    if (c->offload) {
+        if ((rc = check_dev(st->cache, true)) || (rc = check_dev(st->slot_block, false)) ||
+            (rc = check_dev(st->block_slot, false)))
+            return rc;
+    }
+    return NOSA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// Tensor map over a block-major KV buffer seen as [rows][128] bf16 rows,
+// box = 64 rows x 64 dims (128 bytes), 128-byte swizzle.
+int kv_tensor_map(CUtensorMap *map, const void *base, int64_t rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (!enc) return NOSA_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kRowBytes};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NOSA_OK : NOSA_ERR_CUDA;
+}
+
+int select_nchunks(const nosa_config *c, const Geo &g) {
+    if (c->k_q <= 0) return 1;
+    const int cb = select_chunk_blocks((int32_t)g.units, (int32_t)g.nblk);
+    int64_t n = (g.nblk - 1 + cb - 1) / cb;
+    return n < 1 ? 1 : (int)n;
+}
+
+size_t ws_bytes_of(const nosa_config *c, int which) {
+    Geo g;
+    if (!geo_of(c, &g)) return 0;
+    const size_t counters = align256((size_t)g.units * sizeof(int32_t));
+    if (which == NOSA_WS_SELECT) {
+        const int n = select_nchunks(c, g);
+        return n > 1 ? counters + (size_t)g.units * n * 32 * sizeof(uint64_t) : 0;
+    }
+    if (which == NOSA_WS_SPARSE_DECODE || which == NOSA_WS_DENSE_DECODE) {
+        const int n = decode_chunks((int32_t)g.units,
+                                    (int32_t)(which == NOSA_WS_SPARSE_DECODE ? g.max_sel : g.nblk));
+        return n > 1 ? counters + (size_t)g.units * n * kPartFloats * sizeof(float) : 0;
+    }
+    return 0;
+}
+
+int check_ws(const nosa_config *c, int which, void *ws, size_t ws_bytes) {
+    const size_t need = ws_bytes_of(c, which);
+    if (need == 0) return NOSA_OK;
+    if (!ws || ws_bytes < need) return NOSA_ERR_CAPACITY;
+    return check_dev(ws, true);
+}
+
+int run_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q, const int32_t *sel,
+               const int32_t *nsel, const int32_t *block_table, uint16_t *out, void *ws,
+               size_t ws_bytes, void *stream, bool dense) {
+    Geo g;
+    int rc;
+    if ((rc = nosa_validate_config(c))) return rc;
+    geo_of(c, &g);
+    if ((rc = check_state(c, st))) return rc;
+    if ((rc = check_dev(q, true)) || (rc = check_dev(out, true))) return rc;
+    if (!dense) {
+        if ((rc = check_dev(sel, false)) || (rc = check_dev(nsel, false))) return rc;
+        if (c->offload && (rc = check_dev(block_table, false))) return rc;
+    }
+    const int which = dense ? NOSA_WS_DENSE_DECODE : NOSA_WS_SPARSE_DECODE;
+    if ((rc = check_ws(c, which, ws, ws_bytes))) return rc;
+
+    const void *base;
+    int64_t bpu;
+    if (c->offload) {
+        base = st->cache;
+        bpu = g.nslots;
+    } else {
+        uint8_t *s;
+        if ((rc = store_addr(c, st, &s))) return rc;
+        base = s;
+        bpu = g.nblk;
+    }
+    CUtensorMap map;
+    if ((rc = kv_tensor_map(&map, base, g.units * bpu * 2 * kBlock))) return rc;
+
+    DecodeParams p;
+    memset(&p, 0, sizeof(p));
+    p.q = q;
+    p.sel = dense ? nullptr : sel;
+    p.nsel = dense ? nullptr : nsel;
+    p.block_table = (dense || !c->offload) ? nullptr : block_table;
+    p.e = st->evict_logit;
+    p.seq_len = st->seq_len;
+    p.out = out;
+    p.err = st->err;
+    p.max_ctx = c->max_ctx;
+    p.blocks_per_unit = (int32_t)bpu;
+    p.max_sel = (int32_t)g.max_sel;
+    p.G = (int32_t)g.G;
+    p.units = (int32_t)g.units;
+    p.nchunks = decode_chunks(p.units, (int32_t)(dense ? g.nblk : g.max_sel));
+    p.qk_log2 = c->scale * 1.4426950408889634f;
+    if (p.nchunks > 1) {
+        p.counter = static_cast<int32_t *>(ws);
+        p.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) +
+                                           align256((size_t)g.units * sizeof(int32_t)));
+    }
+    return launch_decode(p, map, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int nosa_validate_config(const nosa_config *c) {
+    if (!c) return NOSA_ERR_ARG;
+    if (c->batch < 1 || c->heads_kv < 1 || c->heads_q < 1 || c->heads_q % c->heads_kv) return NOSA_ERR_ARG;
+    if (c->k_q < 0 || c->k_e < 0 || c->k_q + c->k_e < 1 || c->max_ctx <= 0 ||
+        c->max_ctx % 64 || c->reserved != 0 || !(c->scale > 0.f) || !isfinite(c->scale))
+        return NOSA_ERR_ARG;
+    if (c->offload != 0 && c->offload != 1) return NOSA_ERR_ARG;
+    if (c->head_dim != kD || c->block != kBlock || c->sub_block != kSub || c->local_blocks != 1)
+        return NOSA_ERR_UNSUPPORTED;
+    if (c->heads_q / c->heads_kv > kMaxG || c->k_q > kMaxKq || c->k_e > kMaxKe)
+        return NOSA_ERR_UNSUPPORTED;
+    if (c->max_ctx > kMaxCtx) return NOSA_ERR_CAPACITY;
+    const int64_t units = (int64_t)c->batch * c->heads_kv;
+    const int64_t rows = units * (c->max_ctx / kBlock) * 2 * kBlock;
+    if (rows >= (1ll << 31)) return NOSA_ERR_CAPACITY;
+    return NOSA_OK;
+}
+
+size_t nosa_state_bytes(const nosa_config *c, int which) {
+    Geo g;
+    if (!geo_of(c, &g)) return 0;
+    const size_t u = (size_t)g.units;
+    switch (which) {
+    case NOSA_BUF_KV_STORE: return u * g.nblk * kBlockBytes;
+    case NOSA_BUF_EVICT_LOGIT: return u * c->max_ctx * sizeof(float);
+    case NOSA_BUF_CK: return u * g.nsub * kD * sizeof(float);
+    case NOSA_BUF_BLK_EVICT: return u * g.nblk * sizeof(double);
+    case NOSA_BUF_GAMMA_E: return u * (c->k_e > 0 ? c->k_e : 1) * sizeof(int32_t);
+    case NOSA_BUF_GAMMA_N:
+    case NOSA_BUF_SEQ_LEN: return u * sizeof(int32_t);
+    case NOSA_BUF_CACHE: return c->offload ? u * g.nslots * kBlockBytes : 0;
+    case NOSA_BUF_SLOT_BLOCK: return c->offload ? u * g.nslots * sizeof(int32_t) : 0;
+    case NOSA_BUF_BLOCK_SLOT: return c->offload ? u * g.nblk * sizeof(int32_t) : 0;
+    case NOSA_BUF_ERR: return sizeof(uint32_t);
+    default: return 0;
+    }
+}
+
+size_t nosa_workspace_bytes(const nosa_config *c, int which) { return ws_bytes_of(c, which); }
+
+int nosa_state_init(const nosa_config *c, const nosa_state *st, void *stream) {
+    int rc;
+    if ((rc = nosa_validate_config(c))) return rc;
+    if ((rc = check_state(c, st))) return rc;
+    uint8_t *s;
+    if ((rc = store_addr(c, st, &s))) return rc;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    bool ok = cudaMemsetAsync(st->gamma_n, 0, nosa_state_bytes(c, NOSA_BUF_GAMMA_N), cs) == cudaSuccess &&
+              cudaMemsetAsync(st->seq_len, 0, nosa_state_bytes(c, NOSA_BUF_SEQ_LEN), cs) == cudaSuccess &&
+              cudaMemsetAsync(st->err, 0, sizeof(uint32_t), cs) == cudaSuccess;
+    if (ok && c->offload) {
+        ok = cudaMemsetAsync(st->slot_block, 0xFF, nosa_state_bytes(c, NOSA_BUF_SLOT_BLOCK), cs) == cudaSuccess &&
+             cudaMemsetAsync(st->block_slot, 0xFF, nosa_state_bytes(c, NOSA_BUF_BLOCK_SLOT), cs) == cudaSuccess &&
+             cudaMemsetAsync(st->cache, 0, nosa_state_bytes(c, NOSA_BUF_CACHE), cs) == cudaSuccess;
+    }
+    return ok ? NOSA_OK : NOSA_ERR_CUDA;
+}
+
+int nosa_compress_append(const nosa_config *c, const nosa_state *st, const uint16_t *k_new,
+                         const uint16_t *v_new, const float *e_new, int32_t T, const int32_t *lens,
+                         void *stream) {
+    Geo g;
+    int rc;
+    if ((rc = nosa_validate_config(c))) return rc;
+    geo_of(c, &g);
+    if ((rc = check_state(c, st))) return rc;
+    if (T < 1) return NOSA_ERR_ARG;
+    if (T > c->max_ctx) return NOSA_ERR_CAPACITY;
+    if ((rc = check_dev(k_new, true)) || (rc = check_dev(v_new, true)) || (rc = check_dev(e_new, false)))
+        return rc;
+    if (lens) {
+        if (T == 1) return NOSA_ERR_ARG;
+        if ((rc = check_dev(lens, false))) return rc;
+    }
+    uint8_t *s;
+    if ((rc = store_addr(c, st, &s))) return rc;
+    AppendParams p;
+    memset(&p, 0, sizeof(p));
+    p.k_new = k_new; p.v_new = v_new; p.e_new = e_new; p.lens = lens;
+    p.store = s;
+    p.cache = static_cast<uint8_t *>(c->offload ? st->cache : nullptr);
+    p.e_store = st->evict_logit; p.ck = st->ck; p.blk_evict = st->blk_evict;
+    p.gamma_e = st->gamma_e; p.gamma_n = st->gamma_n; p.seq_len = st->seq_len;
+    p.slot_block = st->slot_block; p.block_slot = st->block_slot; p.err = st->err;
+    p.max_ctx = c->max_ctx;
+    p.nblk = (int32_t)g.nblk; p.nsub = (int32_t)g.nsub; p.nslots = (int32_t)g.nslots;
+    p.units = (int32_t)g.units; p.heads_kv = c->heads_kv; p.k_e = c->k_e;
+    p.offload = c->offload; p.T = T;
+    return launch_append(p, static_cast<cudaStream_t>(stream));
+}
+
+int nosa_select(const nosa_config *c, const nosa_state *st, const uint16_t *q, int32_t *sel,
+                int32_t *nsel, int32_t *gq, void *ws, size_t ws_bytes, void *stream) {
+    Geo g;
+    int rc;
+    if ((rc = nosa_validate_config(c))) return rc;
+    geo_of(c, &g);
+    if ((rc = check_state(c, st))) return rc;
+    if ((rc = check_dev(q, true)) || (rc = check_dev(sel, false)) || (rc = check_dev(nsel, false)))
+        return rc;
+    if (gq && (rc = check_dev(gq, false))) return rc;
+    if ((rc = check_ws(c, NOSA_WS_SELECT, ws, ws_bytes))) return rc;
+    SelectParams p;
+    memset(&p, 0, sizeof(p));
+    p.q = q; p.ck = st->ck; p.gamma_e = st->gamma_e; p.gamma_n = st->gamma_n; p.seq_len = st->seq_len;
+    p.sel = sel; p.nsel = nsel; p.gq = c->k_q > 0 ? gq : nullptr; p.err = st->err;
+    p.nsub = (int32_t)g.nsub; p.nblk = (int32_t)g.nblk; p.G = (int32_t)g.G; p.units = (int32_t)g.units;
+    p.nchunks = select_nchunks(c, g);
+    p.chunk_blocks = c->k_q > 0 ? select_chunk_blocks(p.units, p.nblk) : p.nblk;
+    p.k_q = c->k_q; p.k_e = c->k_e; p.max_sel = (int32_t)g.max_sel; p.scale = c->scale;
+    if (p.nchunks > 1) {
+        p.counter = static_cast<int32_t *>(ws);
+        p.part_keys = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(ws) +
+                                                   align256((size_t)g.units * sizeof(int32_t)));
+    }
+    return launch_select(p, static_cast<cudaStream_t>(stream));
+}
+
+int nosa_cache_sync(const nosa_config *c, const nosa_state *st, const int32_t *sel,
+                    const int32_t *nsel, int32_t *block_table, int32_t *n_fetched, void *stream) {
+    Geo g;
+    int rc;
+    if ((rc = nosa_validate_config(c))) return rc;
+    if (!c->offload) return NOSA_ERR_ARG;
+    geo_of(c, &g);
+    if ((rc = check_state(c, st))) return rc;
+    if ((rc = check_dev(sel, false)) || (rc = check_dev(nsel, false)) ||
+        (rc = check_dev(block_table, false)))
+        return rc;
+    if (n_fetched && (rc = check_dev(n_fetched, false))) return rc;
+    uint8_t *s;
+    if ((rc = store_addr(c, st, &s))) return rc;
+    CacheParams p;
+    memset(&p, 0, sizeof(p));
+    p.sel = sel; p.nsel = nsel; p.store = s; p.cache = static_cast<uint8_t *>(st->cache);
+    p.slot_block = st->slot_block; p.block_slot = st->block_slot; p.block_table = block_table;
+    p.n_fetched = n_fetched; p.err = st->err;
+    p.nblk = (int32_t)g.nblk; p.nslots = (int32_t)g.nslots; p.units = (int32_t)g.units;
+    p.max_sel = (int32_t)g.max_sel;
+    return launch_cache_sync(p, static_cast<cudaStream_t>(stream));
+}
+
+int nosa_sparse_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q,
+                       const int32_t *sel, const int32_t *nsel, const int32_t *block_table,
+                       uint16_t *out, void *ws, size_t ws_bytes, void *stream) {
+    return run_decode(c, st, q, sel, nsel, block_table, out, ws, ws_bytes, stream, false);
+}
+
+int nosa_dense_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q,
+                      uint16_t *out, void *ws, size_t ws_bytes, void *stream) {
+    if (c && c->offload) return NOSA_ERR_ARG;
+    return run_decode(c, st, q, nullptr, nullptr, nullptr, out, ws, ws_bytes, stream, true);
+}
+
+int nosa_read_error(const nosa_state *st, uint32_t *flags, int clear, void *stream) {
+    if (!st || !flags) return NOSA_ERR_ARG;
+    int rc;
+    if ((rc = check_dev(st->err, false))) return rc;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    uint32_t h = 0;
+    if (cudaMemcpyAsync(&h, st->err, sizeof(h), cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+        cudaStreamSynchronize(cs) != cudaSuccess)
+        return NOSA_ERR_CUDA;
+    if (clear && (cudaMemsetAsync(st->err, 0, sizeof(uint32_t), cs) != cudaSuccess ||
+                  cudaStreamSynchronize(cs) != cudaSuccess))
+        return NOSA_ERR_CUDA;
+    *flags = h;
+    return h ? NOSA_ERR_DEVICE : NOSA_OK;
+}
+
+const char *nosa_strerror(int code) {
+    switch (code) {
+    case NOSA_OK: return "ok";
+    case NOSA_ERR_ARG: return "invalid argument";
+    case NOSA_ERR_CAPACITY: return "size exceeds buffer or kernel capacity";
+    case NOSA_ERR_PTR: return "pointer of the wrong memory kind or misaligned";
+    case NOSA_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case NOSA_ERR_TIMEOUT: return "bounded device wait ran out";
+    case NOSA_ERR_UNSUPPORTED: return "configuration not supported by this build";
+    case NOSA_ERR_DEVICE: return "device error word has bits set";
+    default: return "unknown error";
+    }
+}
+
+}  // extern "C"

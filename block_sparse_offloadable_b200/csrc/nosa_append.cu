@@ -1,0 +1,308 @@
+// nosa_append.cu -- step a1: append the new token, pool what completes, keep Gamma_e.
+//
+// NOSA pages: montaan.com summary of arXiv:2510.13602, "Key Design Components"
+// item 2 (mean pooling within sub-blocks and max pooling across them, for the
+// query-aware and the query-agnostic selection), item 1 (a block dropped by
+// the query-agnostic selection is never selected by it again); gist.science
+// summary, "ED-DMA" (selection on the pre-exponential eviction score) and
+// "Systeme : NOSI" (block-sized KV units on both GPU and CPU).
+//
+// Decode (T = 1): one warp per unit.  The only HBM traffic is the new rows
+// (512 B), one 4 KiB re-read of the keys of a sub-block when it completes,
+// and one 256 B read of the eviction logits when a block completes, so the
+// kernel is latency-bound by design.
+#include "nosa_internal.cuh"
+
+namespace nosa {
+
+// Warp-cooperative argmin over Gamma_e by (E ascending, block id descending):
+// the member that leaves when a better block arrives.
+__device__ __forceinline__ void gamma_e_worst(const int32_t *ge, int32_t ne, const double *E,
+                                              int lane, double &wE, int32_t &wid, int32_t &wpos) {
+    wE = __longlong_as_double(0x7FF0000000000000ll);  // +inf
+    wid = -1;
+    wpos = -1;
+    for (int j = lane; j < ne; j += 32) {
+        int32_t id = ge[j];
+        double v = E[id];
+        if (v < wE || (v == wE && id > wid)) { wE = v; wid = id; wpos = j; }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        double oE = __shfl_xor_sync(0xFFFFFFFFu, wE, o);
+        int32_t oid = __shfl_xor_sync(0xFFFFFFFFu, wid, o);
+        int32_t opos = __shfl_xor_sync(0xFFFFFFFFu, wpos, o);
+        bool take = (oid >= 0) && (wid < 0 || oE < wE || (oE == wE && oid > wid));
+        if (take) { wE = oE; wid = oid; wpos = opos; }
+    }
+}
+
+__global__ void __launch_bounds__(128) append_decode_kernel(const AppendParams p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u = blockIdx.x * (blockDim.x >> 5) + warp;
+    if (u >= p.units) return;
+    const int32_t pos = p.seq_len[u];
+    if (pos < 0 || pos >= p.max_ctx) {
+        if (lane == 0) set_error(p.err, NOSA_EFLAG_CAPACITY);
+        return;
+    }
+    const int32_t blk = pos >> 6, w = pos & 63;
+    uint8_t *dst;
+    uint8_t *host = nullptr;
+    if (p.offload) {
+        int32_t slot = -1;
+        if (w == 0) {
+            // A new local block: take the lowest free cache slot (one is always
+            // left free by the previous cache sync).
+            for (int s0 = 0; s0 < p.nslots && slot < 0; s0 += 32) {
+                int s = s0 + lane;
+                bool fr = s < p.nslots && p.slot_block[(int64_t)u * p.nslots + s] < 0;
+                unsigned m = __ballot_sync(0xFFFFFFFFu, fr);
+                if (m) slot = s0 + __ffs(m) - 1;
+            }
+            if (slot < 0) {
+                if (lane == 0) set_error(p.err, NOSA_EFLAG_NOSLOT);
+                return;
+            }
+            if (lane == 0) {
+                p.slot_block[(int64_t)u * p.nslots + slot] = blk;
+                p.block_slot[(int64_t)u * p.nblk + blk] = slot;
+            }
+        } else {
+            slot = p.block_slot[(int64_t)u * p.nblk + blk];
+            if (slot < 0) {
+                if (lane == 0) set_error(p.err, NOSA_EFLAG_STATE);
+                return;
+            }
+        }
+        dst = p.cache + ((int64_t)u * p.nslots + slot) * kBlockBytes;
+        host = p.store + ((int64_t)u * p.nblk + blk) * kBlockBytes;
+    } else {
+        dst = p.store + ((int64_t)u * p.nblk + blk) * kBlockBytes;
+    }
+
+    // new key row (lanes 0-15) and value row (lanes 16-31), 16 B per lane
+    const int chunk = lane & 15;
+    const uint16_t *src = (lane < 16 ? p.k_new : p.v_new) + (int64_t)u * kD;
+    const uint4 val = reinterpret_cast<const uint4 *>(src)[chunk];
+    const int64_t off = (lane < 16 ? 0 : kHalfBlockBytes) + (int64_t)w * kRowBytes + chunk * 16;
+    *reinterpret_cast<uint4 *>(dst + off) = val;
+    if (host) *reinterpret_cast<uint4 *>(host + off) = val;  // write-through over PCIe
+    const float e_tok = p.e_new[u];
+    if (lane == 0) p.e_store[(int64_t)u * p.max_ctx + pos] = e_tok;
+
+    // sub-block complete: its compressed key is the mean of its 16 keys (fp64 sum)
+    if (((pos + 1) & (kSub - 1)) == 0) {
+        const int32_t s = pos >> 4;
+        double acc0 = 0.0, acc1 = 0.0, acc2 = 0.0, acc3 = 0.0;
+        const uint8_t *rows = dst + (int64_t)(w - (kSub - 1)) * kRowBytes + lane * 8;
+        for (int j = 0; j < kSub - 1; ++j) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(rows + (int64_t)j * kRowBytes);
+            acc0 += bf16_lo(v.x); acc1 += bf16_hi(v.x);
+            acc2 += bf16_lo(v.y); acc3 += bf16_hi(v.y);
+        }
+        const uint2 v = reinterpret_cast<const uint2 *>(p.k_new + (int64_t)u * kD)[lane];
+        acc0 += bf16_lo(v.x); acc1 += bf16_hi(v.x);
+        acc2 += bf16_lo(v.y); acc3 += bf16_hi(v.y);
+        float4 out = make_float4((float)(acc0 / kSub), (float)(acc1 / kSub), (float)(acc2 / kSub),
+                                 (float)(acc3 / kSub));
+        reinterpret_cast<float4 *>(p.ck + ((int64_t)u * p.nsub + s) * kD)[lane] = out;
+    }
+
+    // block complete: E_b = max over its sub-blocks of the mean eviction logit (fp64)
+    if (((pos + 1) & (kBlock - 1)) == 0) {
+        double m = -__longlong_as_double(0x7FF0000000000000ll);
+        if (lane < kSubPerBlock) {
+            const float *e = p.e_store + (int64_t)u * p.max_ctx + (int64_t)blk * kBlock + lane * kSub;
+            double acc = 0.0;
+            for (int j = 0; j < kSub; ++j)
+                acc += (double)((lane == kSubPerBlock - 1 && j == kSub - 1) ? e_tok : e[j]);
+            m = acc / kSub;
+        }
+        m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        if (lane == 0) p.blk_evict[(int64_t)u * p.nblk + blk] = m;
+    }
+
+    // the previous local block just became a candidate: offer it to Gamma_e
+    if (w == 0 && blk >= 1 && p.k_e > 0) {
+        const int32_t c = blk - 1;
+        int32_t *ge = p.gamma_e + (int64_t)u * p.k_e;
+        const double *E = p.blk_evict + (int64_t)u * p.nblk;
+        const int32_t ne = p.gamma_n[u];
+        if (ne < p.k_e) {
+            if (lane == 0) {
+                ge[ne] = c;  // c is the largest id: the list stays ascending
+                p.gamma_n[u] = ne + 1;
+            }
+        } else {
+            double wE;
+            int32_t wid, wpos;
+            gamma_e_worst(ge, ne, E, lane, wE, wid, wpos);
+            // c has the highest index, so it loses ties: it must be strictly better
+            if (wid >= 0 && E[c] > wE) {
+                int32_t keep[kMaxKe / 32];
+#pragma unroll
+                for (int i = 0; i < kMaxKe / 32; ++i) {
+                    int j = lane + 32 * i;
+                    keep[i] = (j < ne) ? ((j < wpos) ? ge[j] : (j + 1 < ne ? ge[j + 1] : c)) : -1;
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < kMaxKe / 32; ++i) {
+                    int j = lane + 32 * i;
+                    if (j < ne) ge[j] = keep[i];
+                }
+            }
+        }
+    }
+    if (lane == 0) p.seq_len[u] = pos + 1;
+}
+
+// ---- prefill ----------------------------------------------------------------------
+
+__device__ __forceinline__ int32_t unit_len(const AppendParams &p, int32_t u) {
+    return p.lens ? min(p.lens[u / p.heads_kv], p.T) : p.T;
+}
+
+// Store the rows of every unit (block-major), their eviction logits, and in
+// offload mode the rows of the local block into cache slot 0.  One warp per row.
+__global__ void __launch_bounds__(256) prefill_store_kernel(const AppendParams p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t rows = (int64_t)p.units * p.T;
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+         r += nwarps) {
+        const int32_t u = (int32_t)(r / p.T);
+        const int32_t t = (int32_t)(r - (int64_t)u * p.T);
+        const int32_t len = unit_len(p, u);
+        if (t >= len || p.seq_len[u] != 0) continue;
+        const int32_t blk = t >> 6, w = t & 63;
+        const int chunk = lane & 15;
+        const uint16_t *src = (lane < 16 ? p.k_new : p.v_new) + ((int64_t)u * p.T + t) * kD;
+        const uint4 val = reinterpret_cast<const uint4 *>(src)[chunk];
+        const int64_t off = (lane < 16 ? 0 : kHalfBlockBytes) + (int64_t)w * kRowBytes + chunk * 16;
+        *reinterpret_cast<uint4 *>(p.store + ((int64_t)u * p.nblk + blk) * kBlockBytes + off) = val;
+        if (p.offload && blk == (len - 1) >> 6)
+            *reinterpret_cast<uint4 *>(p.cache + (int64_t)u * p.nslots * kBlockBytes + off) = val;
+        if (lane == 0) p.e_store[(int64_t)u * p.max_ctx + t] = p.e_new[(int64_t)u * p.T + t];
+    }
+}
+
+// Pool every complete sub-block (mean key) and block (eviction score).  One warp per block.
+__global__ void __launch_bounds__(256) prefill_pool_kernel(const AppendParams p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int32_t bpu = (p.T + kBlock - 1) / kBlock;
+    const int64_t items = (int64_t)p.units * bpu;
+    for (int64_t it = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); it < items;
+         it += nwarps) {
+        const int32_t u = (int32_t)(it / bpu);
+        const int32_t blk = (int32_t)(it - (int64_t)u * bpu);
+        const int32_t len = unit_len(p, u);
+        if (p.seq_len[u] != 0) continue;
+        const uint16_t *K = p.k_new + (int64_t)u * p.T * kD;
+        for (int s = 0; s < kSubPerBlock; ++s) {
+            const int32_t t0 = blk * kBlock + s * kSub;
+            if (t0 + kSub > len) break;
+            double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+            for (int j = 0; j < kSub; ++j) {
+                const uint2 v = reinterpret_cast<const uint2 *>(K + (int64_t)(t0 + j) * kD)[lane];
+                a0 += bf16_lo(v.x); a1 += bf16_hi(v.x);
+                a2 += bf16_lo(v.y); a3 += bf16_hi(v.y);
+            }
+            float4 out = make_float4((float)(a0 / kSub), (float)(a1 / kSub), (float)(a2 / kSub),
+                                     (float)(a3 / kSub));
+            reinterpret_cast<float4 *>(p.ck + ((int64_t)u * p.nsub + (t0 >> 4)) * kD)[lane] = out;
+        }
+        if ((blk + 1) * kBlock <= len) {
+            double m = -__longlong_as_double(0x7FF0000000000000ll);
+            if (lane < kSubPerBlock) {
+                const float *e = p.e_new + (int64_t)u * p.T + (int64_t)blk * kBlock + lane * kSub;
+                double acc = 0.0;
+                for (int j = 0; j < kSub; ++j) acc += (double)e[j];
+                m = acc / kSub;
+            }
+            m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            if (lane == 0) p.blk_evict[(int64_t)u * p.nblk + blk] = m;
+        }
+    }
+}
+
+// Gamma_e := top-k_e of the candidates by E (ties to the lower block), ascending.
+// One CTA per unit; rank counting over the candidates held in shared memory.
+__global__ void __launch_bounds__(256) prefill_gamma_kernel(const AppendParams p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int32_t u = blockIdx.x;
+    if (p.seq_len[u] != 0) {
+        if (threadIdx.x == 0) set_error(p.err, NOSA_EFLAG_STATE);
+        return;
+    }
+    const int32_t len = unit_len(p, u);
+    const int32_t nb_c = len > 0 ? (len - 1) / kBlock : 0;
+    double *E = reinterpret_cast<double *>(smem);
+    uint8_t *flag = smem + (size_t)p.nblk * sizeof(double);
+    for (int i = threadIdx.x; i < nb_c; i += blockDim.x) E[i] = p.blk_evict[(int64_t)u * p.nblk + i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb_c; i += blockDim.x) {
+        const double ei = E[i];
+        int32_t rank = 0;
+        for (int j = 0; j < nb_c && rank < p.k_e; ++j) {
+            const double ej = E[j];
+            rank += (ej > ei) || (ej == ei && j < i);
+        }
+        flag[i] = rank < p.k_e;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int32_t per = (nb_c + 31) / 32;
+        const int32_t b0 = min(lane * per, nb_c), b1 = min(b0 + per, nb_c);
+        int32_t cnt = 0;
+        for (int i = b0; i < b1; ++i) cnt += flag[i];
+        int32_t pre = cnt;
+        for (int o = 1; o < 32; o <<= 1) {
+            int32_t v = __shfl_up_sync(0xFFFFFFFFu, pre, o);
+            if (lane >= o) pre += v;
+        }
+        int32_t at = pre - cnt;
+        int32_t *ge = p.gamma_e + (int64_t)u * p.k_e;
+        for (int i = b0; i < b1; ++i)
+            if (flag[i]) ge[at++] = i;
+        if (lane == 31) {
+            p.gamma_n[u] = pre;
+            if (p.offload && len > 0) {
+                const int32_t local = (len - 1) / kBlock;
+                p.slot_block[(int64_t)u * p.nslots] = local;
+                p.block_slot[(int64_t)u * p.nblk + local] = 0;
+            }
+            p.seq_len[u] = len;
+        }
+    }
+}
+
+int launch_append(const AppendParams &p, cudaStream_t stream) {
+    if (p.T == 1) {
+        const int wpb = 4;
+        append_decode_kernel<<<(p.units + wpb - 1) / wpb, wpb * 32, 0, stream>>>(p);
+        return cudaGetLastError() == cudaSuccess ? NOSA_OK : NOSA_ERR_CUDA;
+    }
+    const int64_t rows = (int64_t)p.units * p.T;
+    int64_t g = (rows + 7) / 8;
+    if (g > 148 * 16) g = 148 * 16;
+    prefill_store_kernel<<<(unsigned)g, 256, 0, stream>>>(p);
+    const int64_t items = (int64_t)p.units * ((p.T + kBlock - 1) / kBlock);
+    g = (items + 7) / 8;
+    if (g > 148 * 16) g = 148 * 16;
+    prefill_pool_kernel<<<(unsigned)g, 256, 0, stream>>>(p);
+    const size_t smem = (size_t)p.nblk * (sizeof(double) + 1);
+    if (smem > 48 * 1024) {
+        if (cudaFuncSetAttribute(prefill_gamma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return NOSA_ERR_CUDA;
+    }
+    prefill_gamma_kernel<<<p.units, 256, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? NOSA_OK : NOSA_ERR_CUDA;
+}
+
+}  // namespace nosa

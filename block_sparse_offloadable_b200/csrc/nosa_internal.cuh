@@ -1,0 +1,86 @@
+// nosa_internal.cuh -- kernel parameter blocks and launchers shared by the
+// libnosa translation units (not part of the C ABI).
+#pragma once
+
+#include "nosa_common.cuh"
+
+namespace nosa {
+
+struct AppendParams {
+    const uint16_t *k_new;   // [u][T][D]
+    const uint16_t *v_new;   // [u][T][D]
+    const float *e_new;      // [u][T]
+    const int32_t *lens;     // [B] or null (prefill)
+    uint8_t *store;          // device address of the KV store (device memory or mapped host)
+    uint8_t *cache;          // offload cache or null
+    float *e_store;          // [u][max_ctx]
+    float *ck;               // [u][nsub][D]
+    double *blk_evict;       // [u][nblk]
+    int32_t *gamma_e;        // [u][k_e]
+    int32_t *gamma_n;        // [u]
+    int32_t *seq_len;        // [u]
+    int32_t *slot_block;     // [u][nslots]
+    int32_t *block_slot;     // [u][nblk]
+    uint32_t *err;
+    int64_t max_ctx;
+    int32_t nblk, nsub, nslots, units, heads_kv, k_e, offload, T;
+};
+
+struct SelectParams {
+    const uint16_t *q;        // [B][Hq][D]
+    const float *ck;          // [u][nsub][D]
+    const int32_t *gamma_e;   // [u][k_e]
+    const int32_t *gamma_n;   // [u]
+    const int32_t *seq_len;   // [u]
+    int32_t *sel;             // [u][max_sel]
+    int32_t *nsel;            // [u]
+    int32_t *gq;              // [u][k_q] or null
+    uint64_t *part_keys;      // [u][nchunks][32]
+    int32_t *counter;         // [u]
+    uint32_t *err;
+    int32_t nsub, nblk, G, units, nchunks, chunk_blocks, k_q, k_e, max_sel;
+    float scale;
+};
+
+struct CacheParams {
+    const int32_t *sel;       // [u][max_sel]
+    const int32_t *nsel;      // [u]
+    const uint8_t *store;     // device address of the host KV store
+    uint8_t *cache;           // [u][nslots][2][64][D]
+    int32_t *slot_block;      // [u][nslots]
+    int32_t *block_slot;      // [u][nblk]
+    int32_t *block_table;     // [u][max_sel]
+    int32_t *n_fetched;       // [u] or null
+    uint32_t *err;
+    int32_t nblk, nslots, units, max_sel;
+};
+
+struct DecodeParams {
+    const uint16_t *q;          // [B][Hq][D]
+    const int32_t *sel;         // [u][max_sel], or null = every block (dense)
+    const int32_t *nsel;        // [u]
+    const int32_t *block_table; // [u][max_sel] or null (block id addresses the store)
+    const float *e;             // [u][max_ctx]
+    const int32_t *seq_len;     // [u]
+    uint16_t *out;              // [B][Hq][D]
+    float *part;                // [u][nchunks][kPartFloats]
+    int32_t *counter;           // [u]
+    uint32_t *err;
+    int64_t max_ctx;
+    int32_t blocks_per_unit;    // blocks per unit in the tensor-mapped buffer (nblk or nslots)
+    int32_t max_sel, G, units, nchunks;
+    float qk_log2;              // scale * log2(e)
+};
+
+constexpr int kPartFloats = 2 * kMaxG + kMaxG * kD;  // m[8], l[8], o[8][128]
+
+int launch_append(const AppendParams &p, cudaStream_t stream);
+int launch_select(const SelectParams &p, cudaStream_t stream);
+int launch_cache_sync(const CacheParams &p, cudaStream_t stream);
+int launch_decode(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t stream);
+
+// Launch geometry, shared by the launchers and the workspace-size queries.
+int select_chunk_blocks(int32_t units, int32_t nblk);
+int decode_chunks(int32_t units, int32_t max_blocks);
+
+}  // namespace nosa

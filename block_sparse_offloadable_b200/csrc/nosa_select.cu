@@ -1,0 +1,224 @@
+// nosa_select.cu -- steps a2 + a3: two-stage block scores and dual selection.
+//
+// NOSA pages: wmrh.cn NOSA-1B release (two-stage attention: Top-K blocks are
+// chosen with the compressed KV, then attention is exact); montaan.com summary
+// of arXiv:2510.13602, "Key Design Components" item 2 (mean pooling inside
+// sub-blocks, max pooling across them) and item 4 (Equation 7: a query-aware
+// budget k_q and a query-agnostic budget k_e); gist.science summary,
+// "Mecanisme de double selection".
+//
+// Design.  The only large operand is the fp32 compressed-key array of a unit
+// (32 B per token: 4 MiB per unit at 128K context), read once per step: the
+// kernel is a streaming GEMV against q_hat = sum of the group's query heads,
+// bound by HBM bandwidth.  Each CTA owns a contiguous chunk of candidate
+// blocks.  One producer thread streams the chunk into a ring of shared-memory
+// stages with bulk asynchronous copies (cp.async.bulk, completion on
+// mbarriers); consumer warps read 32 sub-block rows per stage with 16-byte
+// shared loads, reduce the 32 partial dot products with a 31-shuffle
+// transpose-reduction (each lane ends with one sub-block), max-pool groups of
+// four lanes to block scores, and keep a warp-wide sorted top-32 list of
+// (score, block) keys.  The per-chunk lists go to the workspace; the last CTA
+// of the unit to finish (atomic counter, no waiting) merges them into Gamma_q,
+// forms the union with Gamma_e through a block bitmap, appends the local block
+// and writes the ascending selection.
+#include "nosa_internal.cuh"
+
+namespace nosa {
+
+namespace {
+constexpr int kSelW = 4;    // consumer warps
+constexpr int kSelS = 4;    // stages
+constexpr int kSelSB = 8;   // blocks per stage (32 sub-block rows, 16 KiB)
+constexpr int kStageBytes = kSelSB * kSubPerBlock * kD * 4;
+constexpr int kCtasPerSm = 3;
+
+// One level of the transpose-reduction: lanes exchange the half they do not keep.
+template <int N>
+__device__ __forceinline__ void reduce_level(float (&v)[32], int lane, int o) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const float send = upper ? v[i] : v[i + N];
+        const float keep = upper ? v[i + N] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+    }
+}
+
+size_t select_smem_bytes(int32_t nblk) {
+    return (size_t)kSelS * kStageBytes + kD * sizeof(float) + 2 * kSelS * sizeof(uint64_t) +
+           kSelW * 32 * sizeof(uint64_t) + ((size_t)nblk / 32 + 1) * sizeof(uint32_t);
+}
+}  // namespace
+
+int select_chunk_blocks(int32_t units, int32_t nblk) {
+    int64_t target = 148LL * kCtasPerSm * 2;
+    int64_t per = ((int64_t)units * nblk + target - 1) / target;
+    per = (per + kSelSB - 1) / kSelSB * kSelSB;
+    if (per < kSelSB) per = kSelSB;
+    return (int)per;
+}
+
+__global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t *tiles = smem;
+    float *qhat = reinterpret_cast<float *>(tiles + kSelS * kStageBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(qhat + kD);
+    uint64_t *empty = full + kSelS;
+    uint64_t *lists = empty + kSelS;
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(lists + kSelW * 32);
+    __shared__ int s_last;
+
+    const int32_t u = blockIdx.y, chunk = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int32_t L = p.seq_len[u];
+    const int32_t nb_c = L > 0 ? (L - 1) / kBlock : 0;
+    const int32_t b0 = min(chunk * p.chunk_blocks, nb_c);
+    const int32_t b1 = min(b0 + p.chunk_blocks, nb_c);
+    const int32_t nstage = (p.k_q > 0 && b1 > b0) ? (b1 - b0 + kSelSB - 1) / kSelSB : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kSelS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        fence_mbar_init();
+    }
+    // q_hat = sum of the G query heads of this kv head (their rows are contiguous)
+    for (int d = threadIdx.x; d < kD; d += blockDim.x) {
+        const uint16_t *q = p.q + (int64_t)u * p.G * kD + d;
+        float s = 0.f;
+        for (int h = 0; h < p.G; ++h) s += __uint_as_float((uint32_t)q[h * kD] << 16);
+        qhat[d] = s;
+    }
+    __syncthreads();
+
+    uint64_t list = 0;
+    if (warp == kSelW) {
+        if (lane == 0) {
+            for (int i = 0; i < nstage; ++i) {
+                const int s = i % kSelS;
+                if (i >= kSelS && !mbar_wait(&empty[s], ((i / kSelS) - 1) & 1)) {
+                    set_error(p.err, NOSA_EFLAG_TIMEOUT);
+                    break;
+                }
+                const int32_t bs = b0 + i * kSelSB;
+                const uint32_t bytes = (uint32_t)min(kSelSB, b1 - bs) * (kSubPerBlock * kD * 4);
+                mbar_arrive_expect_tx(&full[s], bytes);
+                bulk_load(tiles + s * kStageBytes,
+                          p.ck + ((int64_t)u * p.nsub + (int64_t)bs * kSubPerBlock) * kD, bytes,
+                          &full[s]);
+            }
+            // never leave with copies in flight
+            for (int i = max(0, nstage - kSelS); i < nstage; ++i)
+                if (!mbar_wait(&full[i % kSelS], (i / kSelS) & 1)) set_error(p.err, NOSA_EFLAG_TIMEOUT);
+        }
+    } else {
+        const float4 qv = reinterpret_cast<const float4 *>(qhat)[lane];
+        for (int i = warp; i < nstage; i += kSelW) {
+            const int s = i % kSelS;
+            if (!mbar_wait(&full[s], (i / kSelS) & 1)) {
+                set_error(p.err, NOSA_EFLAG_TIMEOUT);
+                break;
+            }
+            const uint8_t *t = tiles + s * kStageBytes + lane * 16;
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float4 k = lds128f(t + j * (kD * 4));
+                v[j] = fmaf(qv.w, k.w, fmaf(qv.z, k.z, fmaf(qv.y, k.y, qv.x * k.x)));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            reduce_level<16>(v, lane, 16);
+            reduce_level<8>(v, lane, 8);
+            reduce_level<4>(v, lane, 4);
+            reduce_level<2>(v, lane, 2);
+            reduce_level<1>(v, lane, 1);
+            // lane holds sub-block (bs*4 + lane); max-pool the four sub-blocks of a block
+            float sc = v[0] * p.scale;
+            sc = fmaxf(sc, __shfl_xor_sync(0xFFFFFFFFu, sc, 1));
+            sc = fmaxf(sc, __shfl_xor_sync(0xFFFFFFFFu, sc, 2));
+            const int32_t bs = b0 + i * kSelSB;
+            const int beta = lane >> 2;
+            const uint64_t cand =
+                ((lane & 3) == 0 && bs + beta < b1) ? select_key(sc, bs + beta) : 0ull;
+            list_offer(list, cand, lane);
+        }
+        lists[warp * 32 + lane] = list;
+    }
+    __syncthreads();
+    if (warp != 0) return;
+    for (int w = 1; w < kSelW; ++w) list_offer(list, lists[w * 32 + lane], lane);
+
+    if (p.nchunks > 1) {
+        uint64_t *mine = p.part_keys + ((int64_t)u * p.nchunks + chunk) * 32;
+        mine[lane] = list;
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) s_last = (atomicAdd(&p.counter[u], 1) == p.nchunks - 1);
+        __syncwarp();
+        if (!s_last) return;
+        __threadfence();
+        if (lane == 0) p.counter[u] = 0;
+        list = 0;
+        const uint64_t *all = p.part_keys + (int64_t)u * p.nchunks * 32;
+        for (int c = 0; c < p.nchunks; ++c) list_offer(list, __ldcg(all + c * 32 + lane), lane);
+    }
+
+    // ---- finalize: Gamma_q, union with Gamma_e, local block ----
+    const int32_t myid = (lane < p.k_q && list != 0ull) ? key_block(list) : -1;
+    if (p.gq && lane < p.k_q) p.gq[(int64_t)u * p.k_q + lane] = myid;
+    int32_t *sel = p.sel + (int64_t)u * p.max_sel;
+    if (L <= 0) {
+        for (int i = lane; i < p.max_sel; i += 32) sel[i] = -1;
+        if (lane == 0) p.nsel[u] = 0;
+        return;
+    }
+    const int32_t nw = (nb_c + 31) >> 5;
+    for (int i = lane; i < nw; i += 32) bitmap[i] = 0;
+    __syncwarp();
+    if (myid >= 0) atomicOr(&bitmap[myid >> 5], 1u << (myid & 31));
+    const int32_t ne = min(p.gamma_n[u], p.k_e);
+    const int32_t *ge = p.gamma_e + (int64_t)u * p.k_e;
+    for (int j = lane; j < ne; j += 32) {
+        const int32_t id = ge[j];
+        if (id >= 0 && id < nb_c) atomicOr(&bitmap[id >> 5], 1u << (id & 31));
+    }
+    __syncwarp();
+    const int32_t per = (nw + 31) / 32;
+    const int32_t w0 = min(lane * per, nw), w1 = min(w0 + per, nw);
+    int32_t cnt = 0;
+    for (int i = w0; i < w1; ++i) cnt += __popc(bitmap[i]);
+    int32_t pre = cnt;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t x = __shfl_up_sync(0xFFFFFFFFu, pre, o);
+        if (lane >= o) pre += x;
+    }
+    int32_t at = pre - cnt;
+    for (int i = w0; i < w1; ++i) {
+        uint32_t m = bitmap[i];
+        while (m) {
+            const int bit = __ffs(m) - 1;
+            m &= m - 1;
+            sel[at++] = i * 32 + bit;
+        }
+    }
+    const int32_t total = __shfl_sync(0xFFFFFFFFu, pre, 31);
+    if (lane == 0) {
+        sel[total] = nb_c;  // the local block, (L-1)/64
+        p.nsel[u] = total + 1;
+    }
+    for (int i = total + 1 + lane; i < p.max_sel; i += 32) sel[i] = -1;
+}
+
+int launch_select(const SelectParams &p, cudaStream_t stream) {
+    const size_t smem = select_smem_bytes(p.nblk);
+    if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return NOSA_ERR_CUDA;
+    dim3 grid(p.nchunks, p.units);
+    select_kernel<<<grid, (kSelW + 1) * 32, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? NOSA_OK : NOSA_ERR_CUDA;
+}
+
+}  // namespace nosa

@@ -1,0 +1,262 @@
+/*
+ * nosa.h -- C ABI of libnosa: the per-step decode hot path of NOSA (Native and
+ * Offloadable Sparse Attention, arXiv:2510.13602) on one B200 (sm_100a).
+ *
+ * One decode step of one attention layer is four calls, in this order, on the
+ * same CUDA stream:
+ *   nosa_compress_append  append the new token; pool what completes; update Gamma_e
+ *   nosa_select           two-stage block scores, Gamma_q, union with Gamma_e and local
+ *   nosa_cache_sync       (offload mode) swap blocks: fetch misses host -> device cache
+ *   nosa_sparse_decode    exact softmax attention over the selected blocks
+ * plus nosa_dense_decode, the full-attention comparator.
+ *
+ * Units.  A "unit" is one (sequence b, kv head g) pair, u = b * heads_kv + g.
+ * Blocks are 64 tokens, sub-blocks 16 tokens; block j holds positions
+ * 64j..64j+63.  With L tokens in a unit, blocks 0 .. (L-1)/64 - 1 are the
+ * candidates and block (L-1)/64 is the local block (always kept, never
+ * scored, not counted in k = k_q + k_e).
+ *
+ * Memory.  The caller allocates every buffer (sizes from nosa_state_bytes and
+ * nosa_workspace_bytes).  The library allocates nothing and keeps no state
+ * besides a cached driver entry point.  Every call is asynchronous on the
+ * given stream and validates its arguments on the host before launching
+ * anything; a non-zero return means nothing was launched.  Conditions only
+ * the device can see (a sequence outgrowing max_ctx, a bounded wait running
+ * out) set bits in the device error word (nosa_state.err) and the kernel skips
+ * the affected unit; read them with nosa_read_error.
+ *
+ * Pointers are plain addresses: "device" means device global memory; "host"
+ * means page-locked host memory that the device can address (cudaHostAlloc /
+ * cudaMallocHost, or cudaHostRegister with cudaHostRegisterMapped).  bf16
+ * tensors are passed as uint16_t bit patterns.  Streams are cudaStream_t
+ * values passed as void* (NULL = legacy default stream).
+ */
+#ifndef NOSA_H
+#define NOSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define NOSA_OK 0
+#define NOSA_ERR_ARG (-1)          /* bad argument or inconsistent configuration */
+#define NOSA_ERR_CAPACITY (-2)     /* a size exceeds what the buffers or the kernels hold */
+#define NOSA_ERR_PTR (-3)          /* pointer of the wrong kind or misaligned */
+#define NOSA_ERR_CUDA (-4)         /* a CUDA call or kernel launch failed */
+#define NOSA_ERR_TIMEOUT (-5)      /* reserved: a bounded device wait ran out */
+#define NOSA_ERR_UNSUPPORTED (-6)  /* valid but not built (e.g. head_dim != 128) */
+#define NOSA_ERR_DEVICE (-7)       /* nosa_read_error found device error bits */
+
+/* Device error-word bits (nosa_state.err). */
+#define NOSA_EFLAG_CAPACITY 0x1u   /* append beyond max_ctx: token dropped */
+#define NOSA_EFLAG_TIMEOUT 0x2u    /* a bounded mbarrier wait gave up: output of that tile invalid */
+#define NOSA_EFLAG_NOSLOT 0x4u     /* offload cache had no free slot: token dropped */
+#define NOSA_EFLAG_STATE 0x8u      /* state inconsistent (prefill into a non-empty unit, lost local block) */
+
+/*
+ * Problem configuration.  Built: head_dim 128, block 64, sub_block 16,
+ * local_blocks 1, 1 <= heads_q/heads_kv <= 8, 0 <= k_q <= 32,
+ * 0 <= k_e <= 256, max_ctx a positive multiple of 64 and <= 2^20, and
+ * batch * heads_kv * max_ctx * 2 < 2^31 (tensor-map row coordinates).
+ */
+typedef struct nosa_config {
+    int32_t batch;        /* B sequences */
+    int32_t heads_q;      /* Hq query heads */
+    int32_t heads_kv;     /* Hkv kv heads; G = Hq / Hkv query heads share one kv head */
+    int32_t head_dim;     /* D */
+    int32_t block;        /* tokens per block (64) */
+    int32_t sub_block;    /* tokens per sub-block (16) */
+    int32_t k_q;          /* query-aware budget: Gamma_q = top-k_q blocks by query score */
+    int32_t k_e;          /* query-agnostic budget: Gamma_e = top-k_e blocks by eviction score */
+    int32_t local_blocks; /* local window in blocks (1) */
+    int32_t offload;      /* 0: KV store in device memory; 1: KV store in host memory + device block cache */
+    int64_t max_ctx;      /* capacity in tokens per sequence */
+    float scale;          /* softmax scale of q.k (normally 1/sqrt(D)) */
+    int32_t reserved;     /* must be 0 */
+} nosa_config;
+
+/*
+ * Per-layer state.  Every buffer is caller-owned; nosa_state_bytes(cfg, NOSA_BUF_x)
+ * gives its size.  Layouts (u = unit, nblk = max_ctx/64, nsub = max_ctx/16,
+ * nslots = k_q + k_e + 2):
+ *   kv_store    bf16 [u][nblk][2][64][D]; [..][0] = keys, [..][1] = values.
+ *               Device memory if offload == 0, host memory if offload == 1.
+ *   evict_logit fp32 [u][max_ctx]   per-token eviction logit e_j (device)
+ *   ck          fp32 [u][nsub][D]   compressed keys: mean of each 16-token sub-block (device)
+ *   blk_evict   fp64 [u][nblk]      block eviction score E_b, pre-exponential (device)
+ *   gamma_e     int32 [u][k_e]      Gamma_e block ids, ascending (device)
+ *   gamma_n     int32 [u]           |Gamma_e| (device)
+ *   seq_len     int32 [u]           tokens held, L (device)
+ *   cache       bf16 [u][nslots][2][64][D]  offload block cache (device; NULL if offload == 0)
+ *   slot_block  int32 [u][nslots]   block held by each cache slot, -1 = free (device; offload only)
+ *   block_slot  int32 [u][nblk]     cache slot of each block, -1 = not resident (device; offload only)
+ *   err         uint32 [1]          device error word (device)
+ * nosa_state_init must run once before the first append.
+ */
+typedef struct nosa_state {
+    void *kv_store;
+    float *evict_logit;
+    float *ck;
+    double *blk_evict;
+    int32_t *gamma_e;
+    int32_t *gamma_n;
+    int32_t *seq_len;
+    void *cache;
+    int32_t *slot_block;
+    int32_t *block_slot;
+    uint32_t *err;
+} nosa_state;
+
+enum nosa_buffer {
+    NOSA_BUF_KV_STORE = 0,
+    NOSA_BUF_EVICT_LOGIT,
+    NOSA_BUF_CK,
+    NOSA_BUF_BLK_EVICT,
+    NOSA_BUF_GAMMA_E,
+    NOSA_BUF_GAMMA_N,
+    NOSA_BUF_SEQ_LEN,
+    NOSA_BUF_CACHE,
+    NOSA_BUF_SLOT_BLOCK,
+    NOSA_BUF_BLOCK_SLOT,
+    NOSA_BUF_ERR,
+    NOSA_BUF_COUNT
+};
+
+enum nosa_call { NOSA_WS_SELECT = 0, NOSA_WS_SPARSE_DECODE = 1, NOSA_WS_DENSE_DECODE = 2 };
+
+/* Validate a configuration: NOSA_OK or a negative code. */
+int nosa_validate_config(const nosa_config *cfg);
+
+/* Bytes of one state buffer (0 if the buffer is unused in this mode, or cfg invalid). */
+size_t nosa_state_bytes(const nosa_config *cfg, int which);
+
+/*
+ * Bytes of scratch workspace a call needs (device memory).  A workspace must
+ * be zero-filled once after allocation; every completed call leaves its
+ * counters at zero again, so it can be reused by later calls on the same
+ * stream.  Two calls that overlap on the GPU must not share a workspace.
+ */
+size_t nosa_workspace_bytes(const nosa_config *cfg, int which_call);
+
+/* Reset a state: empty sequences, empty Gamma_e, empty cache, error word 0. */
+int nosa_state_init(const nosa_config *cfg, const nosa_state *st, void *stream);
+
+/*
+ * a1 -- append + compress.  NOSA pages: montaan.com summary of 2510.13602,
+ * "Key Design Components" item 2 (mean pooling within sub-blocks, max pooling
+ * across them, for both selections); gist.science summary, "Mecanisme de
+ * double selection" (Gamma_e and its eviction rule) and "ED-DMA" (the
+ * eviction score stays pre-exponential).
+ *
+ *   k_new, v_new  device bf16 [u][T][D]   keys / values of the appended tokens
+ *   e_new         device fp32 [u][T]      their eviction logits
+ *   T             1 = decode (append one token to every unit);
+ *                 T > 1 = prefill of empty units (every seq_len must be 0)
+ *   lens          device int32 [B] or NULL: prefill only, tokens of sequence b
+ *                 (<= T; ragged batches); NULL = T for every sequence
+ *
+ * For each unit: stores the rows at position L (offload: into the device cache
+ * slot of the local block, and written through to the host store); when a
+ * 16-token sub-block completes, stores its mean key (fp64 sum of the bf16
+ * keys, stored fp32); when a 64-token block completes, stores E_b = max over
+ * its sub-blocks of the mean eviction logit (fp64); when a block becomes a
+ * candidate, it enters Gamma_e if |Gamma_e| < k_e, or replaces the member with
+ * the lowest E if its E is strictly higher (the member is then dropped for
+ * good).  Prefill builds the pooled arrays and Gamma_e = top-k_e by E (ties
+ * to the lower block) and, in offload mode, puts the local block in the cache.
+ * Device errors: NOSA_EFLAG_CAPACITY (L + T > max_ctx; unit skipped),
+ * NOSA_EFLAG_STATE (prefill into a non-empty unit), NOSA_EFLAG_NOSLOT.
+ */
+int nosa_compress_append(const nosa_config *cfg, const nosa_state *st, const uint16_t *k_new,
+                         const uint16_t *v_new, const float *e_new, int32_t T, const int32_t *lens,
+                         void *stream);
+
+/*
+ * a2 + a3 -- two-stage block scoring and dual selection.  NOSA pages:
+ * wmrh.cn NOSA-1B release ("two-stage attention: select Top-K blocks with
+ * compressed KV, then exact attention"); montaan.com items 2 and 4
+ * (Equation 7, the k_q / k_e budgets); gist.science "Mecanisme de double
+ * selection".
+ *
+ *   q      device bf16 [B][Hq][D]  this step's queries
+ *   sel    device int32 [u][k_q+k_e+1] out: S(t) = (Gamma_q U Gamma_e) U {local},
+ *          ascending (the local block, the largest id, last), -1 padded
+ *   nsel   device int32 [u] out: |S(t)|
+ *   gq     device int32 [u][k_q] out or NULL: Gamma_q in rank order, -1 padded
+ *   ws     device workspace of nosa_workspace_bytes(cfg, NOSA_WS_SELECT) bytes
+ *
+ * s_b = max over the four sub-blocks s of b of  (sum over the G query heads h
+ * of kv head g of q_h) . kbar_s * scale, in fp32, for every candidate b;
+ * Gamma_q = the k_q highest (ties to the lower block).  Uses Gamma_e as left
+ * by nosa_compress_append.
+ */
+int nosa_select(const nosa_config *cfg, const nosa_state *st, const uint16_t *q, int32_t *sel,
+                int32_t *nsel, int32_t *gq, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * a4 -- block cache synchronisation (offload mode).  NOSA pages: montaan.com
+ * "System Optimization (NOSI)" item 2 (block-sized KV units on GPU and CPU;
+ * only blocks unused in the current step are swapped out) and item 3 (a
+ * transfer kernel reading host memory directly through UVA); gist.science
+ * "Systeme : NOSI" (set-difference kernels for block swapping).
+ *
+ *   sel, nsel    from nosa_select
+ *   block_table  device int32 [u][k_q+k_e+1] out: cache slot of each sel entry, -1 padded
+ *   n_fetched    device int32 [u] out or NULL: blocks fetched from the host this step
+ *
+ * Frees every slot whose block is not in S(t), assigns the freed slots (in
+ * ascending order) to the blocks of S(t) that are not resident (in ascending
+ * block order), and copies each such block (32 KiB: keys and values) from the
+ * host store into its slot with 16-byte loads through the device mapping of
+ * host memory.  Offload mode only (NOSA_ERR_ARG otherwise).
+ */
+int nosa_cache_sync(const nosa_config *cfg, const nosa_state *st, const int32_t *sel,
+                    const int32_t *nsel, int32_t *block_table, int32_t *n_fetched, void *stream);
+
+/*
+ * a5 -- sparse decode.  NOSA pages: gist.science "ED-DMA" (the exponent of
+ * the eviction score is applied in the attention step) and wmrh.cn (exact
+ * attention over the selected blocks).
+ *
+ *   q            device bf16 [B][Hq][D]
+ *   sel, nsel    from nosa_select
+ *   block_table  device int32 [u][k_q+k_e+1] from nosa_cache_sync (offload), or NULL
+ *                (device store: block ids address the store directly)
+ *   out          device bf16 [B][Hq][D] out
+ *   ws           device workspace of nosa_workspace_bytes(cfg, NOSA_WS_SPARSE_DECODE) bytes
+ *
+ * For every query head h of kv head g: o_h = sum_j p_j v_j with
+ * p = softmax_j(q_h . k_j * scale + e_j) over the tokens j < L of the blocks
+ * in sel; bf16 inputs, fp32 accumulation, bf16 output (round to nearest even).
+ */
+int nosa_sparse_decode(const nosa_config *cfg, const nosa_state *st, const uint16_t *q,
+                       const int32_t *sel, const int32_t *nsel, const int32_t *block_table,
+                       uint16_t *out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * a6 -- dense comparator (FullAttn of the NOSA pages, montaan.com "The
+ * gist"): the same attention, with the same e_j bias, over all L tokens.
+ * Device store only (offload == 0; NOSA_ERR_ARG otherwise).
+ */
+int nosa_dense_decode(const nosa_config *cfg, const nosa_state *st, const uint16_t *q,
+                      uint16_t *out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Read the device error word (synchronises the stream).  *flags receives the
+ * bits; if clear != 0 the word is reset to 0.  Returns NOSA_OK if no bit was
+ * set, NOSA_ERR_DEVICE if some was, or another negative code.
+ */
+int nosa_read_error(const nosa_state *st, uint32_t *flags, int clear, void *stream);
+
+/* Human-readable text of a return code. */
+const char *nosa_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NOSA_H */

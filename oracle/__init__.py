@@ -51,6 +51,7 @@ def lib():
         L.nosa_oracle_E.argtypes = [P]
         L.nosa_oracle_E.restype = ctypes.POINTER(ctypes.c_double)
         L.nosa_oracle_violations.argtypes = [P, P]
+        L.nosa_oracle_attend_blocks.argtypes = [P, P, P, ctypes.c_int32, P]
         _lib = L
     return _lib
 
@@ -114,6 +115,14 @@ class OracleUnit:
         q = np.ascontiguousarray(q, dtype=np.uint16).reshape(self.G, self.D)
         o = np.zeros((self.G, self.D), np.float64)
         lib().nosa_oracle_dense(self._u, _p(q), _p(o))
+        return o
+
+    def attend_blocks(self, q, blocks):
+        """Attention of q [G][D] (bf16 bits) over the tokens of the given blocks."""
+        q = np.ascontiguousarray(q, dtype=np.uint16).reshape(self.G, self.D)
+        b = np.ascontiguousarray(blocks, dtype=np.int32)
+        o = np.zeros((self.G, self.D), np.float64)
+        lib().nosa_oracle_attend_blocks(self._u, _p(q), _p(b), len(b), _p(o))
         return o
 
     @property

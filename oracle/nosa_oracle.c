@@ -411,3 +411,22 @@ void nosa_oracle_violations(const nosa_oracle_unit *u, int64_t out[5]) {
     out[0] = u->viol_gamma; out[1] = u->viol_reselect; out[2] = u->viol_incremental;
     out[3] = u->viol_fetch; out[4] = u->steps;
 }
+
+/*
+ * Attention of the G heads over the tokens (< L) of an arbitrary ascending
+ * block list: used to evaluate the output on another selection (e.g. one that
+ * differs from this unit's by an excused near-tie).
+ */
+int nosa_oracle_attend_blocks(const nosa_oracle_unit *u, const uint16_t *q, const int32_t *blocks,
+                              int32_t n, double *o) {
+    int64_t *tok = (int64_t *)malloc(sizeof(int64_t) * (size_t)(n > 0 ? n : 1) * (size_t)u->block);
+    int64_t n_tok = 0;
+    for (int32_t i = 0; i < n; ++i)
+        for (int32_t j = 0; j < u->block; ++j) {
+            int64_t p = (int64_t)blocks[i] * u->block + j;
+            if (blocks[i] >= 0 && p < u->L) tok[n_tok++] = p;
+        }
+    attend(u, q, tok, n_tok, o);
+    free(tok);
+    return 0;
+}

@@ -21,6 +21,11 @@ def _has_gpu():
         return False
 
 
+def pytest_sessionstart(session):
+    import block_sparse_offloadable_b200 as nosa
+    nosa.build()
+
+
 def pytest_collection_modifyitems(config, items):
     if _has_gpu():
         return

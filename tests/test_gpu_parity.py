@@ -1,0 +1,57 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on small
+seeded workloads that span several tiles, cross block boundaries and have
+ragged tails.  Tolerances: see tests/gpu_harness.py."""
+import pytest
+
+from tests import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(sc, allow_excused=True):
+    data = H.unit_data(sc)
+    gpu = H.run_gpu(sc, data)
+    assert gpu["err"] == 0
+    bad = []
+    st = H.compare(sc, data, gpu, report=bad)
+    assert not bad, bad[:3]
+    H.assert_parity(st, allow_excused)
+    return st
+
+
+def test_gqa8_device_store():
+    _run(H.Scenario(B=2, Hq=16, Hkv=2, k_q=4, k_e=12, L0=64 * 37 + 21, steps=70, seed=1))
+
+
+def test_mha_block_boundary_first_step():
+    _run(H.Scenario(B=1, Hq=4, Hkv=4, k_q=4, k_e=12, L0=64 * 20, steps=66, seed=2))
+
+
+def test_offload_fetch_counts():
+    st = _run(H.Scenario(B=2, Hq=8, Hkv=2, k_q=4, k_e=12, L0=64 * 40 + 3, steps=70, offload=True, seed=3))
+    assert st["fetch_cmp"] > 0
+
+
+@pytest.mark.parametrize("offload", [False, True])
+def test_empty_start_no_prefill(offload):
+    _run(H.Scenario(B=1, Hq=4, Hkv=2, k_q=2, k_e=6, L0=0, steps=150, offload=offload, seed=4))
+
+
+@pytest.mark.parametrize("offload", [False, True])
+def test_ragged_prefill(offload):
+    _run(H.Scenario(B=3, Hq=8, Hkv=2, k_q=4, k_e=8, L0=0, lens=[37, 64 * 9, 64 * 30 + 5], steps=40,
+                    offload=offload, seed=5))
+
+
+def test_dense_decode():
+    _run(H.Scenario(B=2, Hq=16, Hkv=2, k_q=4, k_e=12, L0=64 * 25 + 7, steps=4, seed=6, dense=True))
+
+
+@pytest.mark.parametrize("k_q,k_e", [(32, 96), (0, 16), (16, 0)])
+def test_budget_limits(k_q, k_e):
+    _run(H.Scenario(B=1, Hq=16, Hkv=2, k_q=k_q, k_e=k_e, L0=64 * 300 + 11, steps=6, seed=7))
+
+
+def test_all_blocks_fit_in_budget():
+    # fewer candidates than k: every block selected, sparse == dense
+    _run(H.Scenario(B=2, Hq=8, Hkv=1, k_q=16, k_e=48, L0=64 * 10 + 30, steps=5, seed=8, dense=True))

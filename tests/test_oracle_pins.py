@@ -210,3 +210,16 @@ def test_first_token_and_tiny_context():
     r = u.step(K[0], V[0], float(e[0]), q)
     assert r["sel"].tolist() == [0] and r["nb_c"] == 0
     np.testing.assert_array_equal(r["o"], np.repeat(cases.bf16_bits_to_f64(V[0])[None], 2, 0))
+
+
+def test_attend_blocks_matches_own_selection():
+    L0 = 64 * 30 + 9
+    K, V, e = cases.synthetic_unit(21, 0, 0, 0, L0 + 1)
+    q = cases.synthetic_queries(21, 0, 0, 0, 2, 1)[0]
+    u = OracleUnit(G=2, k_q=3, k_e=5, cap=4096)
+    u.prefill(K[:L0], V[:L0], e[:L0])
+    r = u.step(K[L0], V[L0], float(e[L0]), q)
+    np.testing.assert_array_equal(u.attend_blocks(q, r["sel"]), r["o"])
+    tok = np.concatenate([np.arange(b * 64, b * 64 + 64) for b in (2, 7)])
+    want = cases.textbook_attention(q, K, V, e, tok, 1 / np.sqrt(128))
+    np.testing.assert_allclose(u.attend_blocks(q, [2, 7]), want, rtol=1e-12, atol=1e-15)
