@@ -187,7 +187,9 @@ int run_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q, co
     p.max_sel = (int32_t)g.max_sel;
     p.G = (int32_t)g.G;
     p.units = (int32_t)g.units;
-    p.nchunks = decode_chunks(p.units, (int32_t)(dense ? g.nblk : g.max_sel));
+    const int32_t max_blocks = (int32_t)(dense ? g.nblk : g.max_sel);
+    p.nchunks = decode_chunks(p.units, max_blocks);
+    p.max_nb = (max_blocks + p.nchunks - 1) / p.nchunks + 1;
     p.qk_log2 = c->scale * 1.4426950408889634f;
     if (p.nchunks > 1) {
         p.counter = static_cast<int32_t *>(ws);

@@ -6,10 +6,12 @@
 // (exact attention over the Top-K blocks plus the current window).
 //
 // Design (split-K flash decoding with GQA sharing, per unit = (seq, kv head)):
-//  * grid = (chunks, units); a CTA takes a balanced, contiguous range of the
+//  * grid = (chunks, units), the chunk count chosen against wave quantisation;
+//    a CTA takes a balanced, contiguous range of the
 //    unit's selected blocks (or of all blocks for the dense comparator).
 //  * One producer thread streams every selected block (keys + values, 32 KiB,
-//    plus its 64 eviction logits) into a 4-stage shared-memory ring: four
+//    plus its 64 eviction logits) into a 3-stage shared-memory ring (two CTAs
+//    per SM, so six blocks in flight per SM): four
 //    2-D TMA tile loads (64 rows x 64 dims, 128-byte swizzle) and one bulk
 //    copy per block, completing on the stage's mbarrier.
 //  * Four consumer warps each own 16 of the block's 64 tokens.  S^T = K Q^T is
@@ -33,16 +35,18 @@ namespace nosa {
 
 namespace {
 constexpr int kDecW = 4;                  // consumer warps (16 tokens each)
-constexpr int kDecS = 4;                  // ring stages (one block each)
+constexpr int kDecS = 3;                  // ring stages (one block each); two CTAs per SM
 constexpr int kBoxBytes = 64 * 128;       // one TMA box: 64 rows x 64 bf16
 constexpr int kDecThreads = (kDecW + 1) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kNegInf = -__builtin_huge_valf();
-constexpr int kCtaPerSm = 1;
+constexpr int kCtaPerSm = 2;
 
-size_t decode_smem_bytes() {
+// Every consumer warp consumes every stage, in order, so mbarrier waiters see
+// their phases in order (parity waits cannot tell phase p from p + 2).
+size_t decode_smem_bytes(int32_t max_nb) {
     return 1024 + (size_t)kDecS * kBlockBytes + (size_t)kDecS * kBlock * sizeof(float) +
-           2 * kDecS * sizeof(uint64_t) + kDecS * sizeof(int32_t);
+           2 * kDecS * sizeof(uint64_t) + kDecS * sizeof(int32_t) + 2 * (size_t)max_nb * sizeof(int32_t);
 }
 
 __device__ __forceinline__ uint32_t word(const uint4 &v, int i) {
@@ -51,15 +55,11 @@ __device__ __forceinline__ uint32_t word(const uint4 &v, int i) {
 }  // namespace
 
 int decode_chunks(int32_t units, int32_t max_blocks) {
-    int64_t target = 148LL * kCtaPerSm * 2;
-    int64_t n = (target + units - 1) / units;
-    int64_t cap = max_blocks / 4;
-    if (n > cap) n = cap;
-    if (n < 1) n = 1;
-    return (int)n;
+    // per-CTA fixed cost ~ 3 blocks (first TMA round trip, the partial merge)
+    return best_chunks(units, max_blocks, (int64_t)kNumSms * kCtaPerSm, 3, max_blocks / 4);
 }
 
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, kCtaPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *tiles = reinterpret_cast<uint8_t *>(
@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     uint64_t *full = reinterpret_cast<uint64_t *>(ebuf + kDecS * kBlock);
     uint64_t *empty = full + kDecS;
     int32_t *s_blk = reinterpret_cast<int32_t *>(empty + kDecS);
+    int32_t *s_lid = s_blk + kDecS;         // this CTA's logical block ids
+    int32_t *s_pid = s_lid + p.max_nb;      // and their physical (store or cache) blocks
     __shared__ int s_last;
 
     const int32_t u = blockIdx.y, chunk = blockIdx.x;
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (L <= 0 || nblocks < 0) nblocks = 0;
     const int32_t i0 = (int32_t)((int64_t)chunk * nblocks / p.nchunks);
     const int32_t i1 = (int32_t)((int64_t)(chunk + 1) * nblocks / p.nchunks);
-    const int32_t nb = i1 - i0;
+    const int32_t nb = min(i1 - i0, p.max_nb);  // i1 - i0 <= ceil(max blocks / nchunks) < max_nb
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDecS; ++s) {
@@ -91,18 +93,28 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
     if (warp == kDecW) {
         // ---------------- producer ----------------
-        if (lane == 0) {
+        // fetch the CTA's block ids once, 32 at a time, so no global load sits
+        // between consecutive TMA issues
+        {
             const int32_t *selu = p.sel ? p.sel + (int64_t)u * p.max_sel : nullptr;
             const int32_t *btu = p.block_table ? p.block_table + (int64_t)u * p.max_sel : nullptr;
+            for (int i = lane; i < nb; i += 32) {
+                const int32_t idx = i0 + i;
+                const int32_t lb = selu ? selu[idx] : idx;
+                s_lid[i] = lb;
+                s_pid[i] = btu ? btu[idx] : lb;
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
             for (int i = 0; i < nb; ++i) {
                 const int s = i % kDecS;
                 if (i >= kDecS && !mbar_wait(&empty[s], ((i / kDecS) - 1) & 1)) {
                     set_error(p.err, NOSA_EFLAG_TIMEOUT);
                     break;
                 }
-                const int32_t idx = i0 + i;
-                const int32_t lb = selu ? selu[idx] : idx;
-                const int32_t pb = btu ? btu[idx] : lb;
+                const int32_t lb = s_lid[i];
+                const int32_t pb = s_pid[i];
                 const bool ok = lb >= 0 && (int64_t)lb * kBlock < p.max_ctx && pb >= 0 &&
                                 pb < p.blocks_per_unit;
                 s_blk[s] = ok ? lb : -1;
@@ -159,7 +171,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             if (lb >= 0) {
                 const uint8_t *t = tiles + s * kBlockBytes;
                 // ---- S^T (16 tokens x 8 heads) = K Q^T ----
+                // two independent accumulation chains halve the serial mma latency
                 float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+                float sacc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const uint8_t *box = t + (j >> 1) * kBoxBytes;
@@ -169,8 +183,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     const uint32_t a0[4] = {ka.x, kb.x, ka.y, kb.y};
                     const uint32_t a1[4] = {ka.z, kb.z, ka.w, kb.w};
                     mma_16816(sacc, a0, qf[2 * j]);
-                    mma_16816(sacc, a1, qf[2 * j + 1]);
+                    mma_16816(sacc2, a1, qf[2 * j + 1]);
                 }
+#pragma unroll
+                for (int x = 0; x < 4; ++x) sacc[x] += sacc2[x];
                 // ---- online softmax over this block's 16 tokens, per head (2c, 2c+1) ----
                 const float *eb = ebuf + s * kBlock;
                 const int64_t posA = (int64_t)lb * kBlock + rowA, posB = posA + 8;
@@ -320,7 +336,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 }
 
 int launch_decode(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t stream) {
-    const size_t smem = decode_smem_bytes();
+    const size_t smem = decode_smem_bytes(p.max_nb);
     if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return NOSA_ERR_CUDA;

@@ -69,6 +69,7 @@ struct DecodeParams {
     int64_t max_ctx;
     int32_t blocks_per_unit;    // blocks per unit in the tensor-mapped buffer (nblk or nslots)
     int32_t max_sel, G, units, nchunks;
+    int32_t max_nb;             // upper bound on blocks per CTA: ceil(max blocks / nchunks) + 1
     float qk_log2;              // scale * log2(e)
 };
 
@@ -82,5 +83,21 @@ int launch_decode(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t s
 // Launch geometry, shared by the launchers and the workspace-size queries.
 int select_chunk_blocks(int32_t units, int32_t nblk);
 int decode_chunks(int32_t units, int32_t max_blocks);
+
+constexpr int kNumSms = 148;
+
+// Split each unit's `work` items into n chunks (one CTA each) to minimise the
+// wave-quantised time  ceil(units*n / slots) * (ceil(work/n) + ovh), where
+// `slots` CTAs run at once and `ovh` is the per-CTA fixed cost in work items.
+inline int best_chunks(int64_t units, int64_t work, int64_t slots, int64_t ovh, int64_t nmax) {
+    if (nmax < 1) nmax = 1;
+    int64_t best_n = 1, best_cost = -1;
+    for (int64_t n = 1; n <= nmax; ++n) {
+        const int64_t waves = (units * n + slots - 1) / slots;
+        const int64_t cost = waves * ((work + n - 1) / n + ovh);
+        if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_n = n; }
+    }
+    return (int)best_n;
+}
 
 }  // namespace nosa

@@ -31,6 +31,10 @@ constexpr int kSelS = 4;    // stages
 constexpr int kSelSB = 8;   // blocks per stage (32 sub-block rows, 16 KiB)
 constexpr int kStageBytes = kSelSB * kSubPerBlock * kD * 4;
 constexpr int kCtasPerSm = 3;
+// Stage s is always consumed by warp s % kSelW, so every mbarrier waiter waits
+// its phases in order (parity waits cannot tell phase p from p + 2).
+static_assert(kSelS % kSelW == 0, "each stage must have a single consumer warp");
+constexpr int kMaxChunks = 64;  // select_chunk_blocks keeps chunks per unit below this
 
 // One level of the transpose-reduction: lanes exchange the half they do not keep.
 template <int N>
@@ -45,24 +49,27 @@ __device__ __forceinline__ void reduce_level(float (&v)[32], int lane, int o) {
 }
 
 size_t select_smem_bytes(int32_t nblk) {
-    return (size_t)kSelS * kStageBytes + kD * sizeof(float) + 2 * kSelS * sizeof(uint64_t) +
+    return (size_t)kSelS * kStageBytes + 2 * kSelS * sizeof(uint64_t) +
            kSelW * 32 * sizeof(uint64_t) + ((size_t)nblk / 32 + 1) * sizeof(uint32_t);
 }
 }  // namespace
 
 int select_chunk_blocks(int32_t units, int32_t nblk) {
-    int64_t target = 148LL * kCtasPerSm * 2;
-    int64_t per = ((int64_t)units * nblk + target - 1) / target;
+    // candidates per unit are at most nblk - 1; per-CTA fixed cost ~ 16 blocks
+    // (pipeline fill and the list merge)
+    const int64_t work = nblk > 1 ? nblk - 1 : 1;
+    int64_t nmax = (work + kSelSB - 1) / kSelSB;
+    if (nmax > kMaxChunks) nmax = kMaxChunks;
+    const int n = best_chunks(units, work, (int64_t)kNumSms * kCtasPerSm, 16, nmax);
+    int64_t per = (work + n - 1) / n;
     per = (per + kSelSB - 1) / kSelSB * kSelSB;
-    if (per < kSelSB) per = kSelSB;
     return (int)per;
 }
 
 __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *tiles = smem;
-    float *qhat = reinterpret_cast<float *>(tiles + kSelS * kStageBytes);
-    uint64_t *full = reinterpret_cast<uint64_t *>(qhat + kD);
+    uint64_t *full = reinterpret_cast<uint64_t *>(tiles + kSelS * kStageBytes);
     uint64_t *empty = full + kSelS;
     uint64_t *lists = empty + kSelS;
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(lists + kSelW * 32);
@@ -82,13 +89,6 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
             mbar_init(&empty[s], 1);
         }
         fence_mbar_init();
-    }
-    // q_hat = sum of the G query heads of this kv head (their rows are contiguous)
-    for (int d = threadIdx.x; d < kD; d += blockDim.x) {
-        const uint16_t *q = p.q + (int64_t)u * p.G * kD + d;
-        float s = 0.f;
-        for (int h = 0; h < p.G; ++h) s += __uint_as_float((uint32_t)q[h * kD] << 16);
-        qhat[d] = s;
     }
     __syncthreads();
 
@@ -113,7 +113,22 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
                 if (!mbar_wait(&full[i % kSelS], (i / kSelS) & 1)) set_error(p.err, NOSA_EFLAG_TIMEOUT);
         }
     } else {
-        const float4 qv = reinterpret_cast<const float4 *>(qhat)[lane];
+        // q_hat = sum of the G query heads of this kv head, lane's 4 dims; the
+        // loads are issued together while the first stages are in flight
+        float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
+        {
+            const uint2 *q = reinterpret_cast<const uint2 *>(p.q + (int64_t)u * p.G * kD) + lane;
+            uint2 w[kMaxG];
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h) w[h] = (h < p.G) ? q[h * (kD / 4)] : make_uint2(0u, 0u);
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h) {
+                if (h < p.G) {
+                    qv.x += bf16_lo(w[h].x); qv.y += bf16_hi(w[h].x);
+                    qv.z += bf16_lo(w[h].y); qv.w += bf16_hi(w[h].y);
+                }
+            }
+        }
         for (int i = warp; i < nstage; i += kSelW) {
             const int s = i % kSelS;
             if (!mbar_wait(&full[s], (i / kSelS) & 1)) {
@@ -162,7 +177,13 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
         if (lane == 0) p.counter[u] = 0;
         list = 0;
         const uint64_t *all = p.part_keys + (int64_t)u * p.nchunks * 32;
-        for (int c = 0; c < p.nchunks; ++c) list_offer(list, __ldcg(all + c * 32 + lane), lane);
+        for (int c0 = 0; c0 < p.nchunks; c0 += 8) {
+            uint64_t k[8];  // issue the loads together, then merge
+#pragma unroll
+            for (int j = 0; j < 8; ++j) k[j] = (c0 + j < p.nchunks) ? __ldcg(all + (c0 + j) * 32 + lane) : 0ull;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) list_offer(list, k[j], lane);
+        }
     }
 
     // ---- finalize: Gamma_q, union with Gamma_e, local block ----
