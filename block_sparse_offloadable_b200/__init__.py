@@ -19,7 +19,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _ROOT = os.path.dirname(_HERE)
 LIB_PATH = os.path.join(_HERE, "_lib", "libnosa.so")
-_SOURCES = ["nosa_api.cu", "nosa_append.cu", "nosa_select.cu", "nosa_cache.cu", "nosa_decode.cu"]
+_SOURCES = ["nosa_api.cu", "nosa_append.cu", "nosa_select.cu", "nosa_cache.cu", "nosa_decode.cu", "nosa_noalloc.cu"]
 _HEADERS = ["nosa_common.cuh", "nosa_internal.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared"]
@@ -33,7 +33,8 @@ WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE = 0, 1, 2
 # Every extern "C" symbol include/nosa.h declares.
 EXPORTS = ["nosa_validate_config", "nosa_state_bytes", "nosa_workspace_bytes", "nosa_state_init",
            "nosa_compress_append", "nosa_select", "nosa_cache_sync", "nosa_sparse_decode",
-           "nosa_dense_decode", "nosa_read_error", "nosa_strerror"]
+           "nosa_dense_decode", "nosa_read_error", "nosa_strerror", "nosa_select_noalloc"]
+NOALLOC_SELECT_SCRATCH = 2 << 20
 
 
 def build(force=False, verbose=False):
@@ -87,6 +88,7 @@ def lib():
         L.nosa_sparse_decode.argtypes = [C, S, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_dense_decode.argtypes = [C, S, P, P, P, ctypes.c_size_t, P]
         L.nosa_read_error.argtypes = [S, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P]
+        L.nosa_select_noalloc.argtypes = [C, S, P, P, P, P, P]
         L.nosa_strerror.argtypes = [ctypes.c_int]
         L.nosa_strerror.restype = ctypes.c_char_p
         _lib = L
@@ -147,6 +149,12 @@ def nosa_select(cfg, st, q, sel, nsel, gq=None, ws=None, stream=None):
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib().nosa_select(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(sel), _ptr(nsel), _ptr(gq), _ptr(ws),
                              nbytes, _stream(stream)), "nosa_select")
+
+
+def nosa_select_noalloc(cfg, st, q, sel, nsel, gq=None, stream=None):
+    """nosa_select with its scratch in the library's fixed device array (allocates nothing)."""
+    _check(lib().nosa_select_noalloc(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(sel), _ptr(nsel), _ptr(gq),
+                                     _stream(stream)), "nosa_select_noalloc")
 
 
 def nosa_cache_sync(cfg, st, sel, nsel, block_table, n_fetched=None, stream=None):

@@ -252,6 +252,29 @@ int nosa_dense_decode(const nosa_config *cfg, const nosa_state *st, const uint16
  */
 int nosa_read_error(const nosa_state *st, uint32_t *flags, int clear, void *stream);
 
+/*
+ * nosa_select without a caller-provided workspace, for callers that cannot
+ * allocate device memory (a plug-in that is handed only its inputs and
+ * outputs, or a path that must not call cudaMalloc because it may
+ * synchronise the device).  The NOSA paper has no counterpart of this entry
+ * point; it exists for such integrations.
+ *
+ * Same arguments, outputs and results as nosa_select, minus ws/ws_bytes.  The
+ * scratch lives in a fixed __device__ array of NOSA_NOALLOC_SELECT_SCRATCH
+ * bytes inside the library (every GPU that loads the library holds it until
+ * the process exits); configurations whose nosa_workspace_bytes(cfg,
+ * NOSA_WS_SELECT) exceeds that size are rejected with NOSA_ERR_CAPACITY.  The
+ * function allocates nothing.  Its first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress, that device current); make
+ * that first call before any stream capture.  Each call clears the array's
+ * counters on the stream before the kernel.  All calls on a device share the
+ * one array, which keeps the last call's contents: calls that overlap on the
+ * GPU (other streams, other threads) race and must not be issued.
+ */
+#define NOSA_NOALLOC_SELECT_SCRATCH (2u << 20)
+int nosa_select_noalloc(const nosa_config *cfg, const nosa_state *st, const uint16_t *q,
+                        int32_t *sel, int32_t *nsel, int32_t *gq, void *stream);
+
 /* Human-readable text of a return code. */
 const char *nosa_strerror(int code);
 

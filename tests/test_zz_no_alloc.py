@@ -1,0 +1,58 @@
+"""nosa_select_noalloc: the select step for callers that cannot allocate device
+memory (its scratch is a fixed array inside the library).  Its results must be
+the same as nosa_select's with a caller-provided workspace, on two calls in a
+row (the second call finds the first call's leftovers in the shared array).
+
+Kept in its own file, collected last, so that a failure here comes after every
+other test has run.  Must pass alone in a fresh process and after the others."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_offloadable_b200 as nosa
+from tests import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,k_q,k_e,L0", [(4, 16, 2, 16, 48, 64 * 300 + 17), (2, 8, 8, 8, 24, 64 * 90 + 63)])
+def test_noalloc_select_matches_workspace_select(B, Hq, Hkv, k_q, k_e, L0):
+    sc = H.Scenario(B=B, Hq=Hq, Hkv=Hkv, k_q=k_q, k_e=k_e, L0=L0, steps=2, seed=31)
+    cfg = sc.cfg()
+    need = nosa.nosa_workspace_bytes(cfg, nosa.WS_SELECT)
+    assert 0 < need <= nosa.NOALLOC_SELECT_SCRATCH  # the case really uses scratch
+    K, V, E, Q = H.unit_data(sc)
+    lay = nosa.NosaLayer(cfg)
+    lay.append(H._dev16(K[:, :L0]), H._dev16(V[:, :L0]), torch.from_numpy(np.ascontiguousarray(E[:, :L0])).cuda(), L0)
+    sel2 = torch.full_like(lay.sel, -7)
+    nsel2 = torch.full_like(lay.nsel, -7)
+    gq2 = torch.full_like(lay.gq, -7)
+    for t in range(2):
+        idx = np.arange(sc.units)
+        lay.append(H._dev16(K[idx, L0 + t][:, None, :]), H._dev16(V[idx, L0 + t][:, None, :]),
+                   torch.from_numpy(np.ascontiguousarray(E[idx, L0 + t][:, None])).cuda(), 1)
+        q = H._dev16(Q[t])
+        lay.select(q)  # the existing entry point, workspace from the caller
+        for _ in range(2):  # two calls in a row on the shared scratch array
+            sel2.fill_(-7), nsel2.fill_(-7), gq2.fill_(-7)
+            nosa.nosa_select_noalloc(cfg, lay.state, q, sel2, nsel2, gq2)
+            torch.cuda.synchronize()
+            assert torch.equal(nsel2, lay.nsel)
+            assert torch.equal(sel2, lay.sel)
+            assert torch.equal(gq2, lay.gq)
+    assert lay.read_error() == 0
+
+
+def test_noalloc_rejects_oversize_workspace():
+    # 8192 (sequence, kv head) units need more select scratch than the fixed array holds;
+    # the call is refused before anything is touched or launched
+    cfg = nosa.make_config(4096, 16, 2, 32, 32, 64000)
+    assert nosa.nosa_validate_config(cfg) == nosa.OK
+    assert nosa.nosa_workspace_bytes(cfg, nosa.WS_SELECT) > nosa.NOALLOC_SELECT_SCRATCH
+    q = torch.zeros(16, dtype=torch.int16, device="cuda")
+    sel = torch.zeros(16, dtype=torch.int32, device="cuda")
+    nsel = torch.zeros(16, dtype=torch.int32, device="cuda")
+    st = nosa.State()
+    with pytest.raises(nosa.NosaError) as ei:
+        nosa.nosa_select_noalloc(cfg, st, q, sel, nsel)
+    assert ei.value.code == nosa.ERR_CAPACITY
