@@ -34,7 +34,7 @@ WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE = 0, 1, 2
 EXPORTS = ["nosa_validate_config", "nosa_state_bytes", "nosa_workspace_bytes", "nosa_state_init",
            "nosa_compress_append", "nosa_select", "nosa_cache_sync", "nosa_sparse_decode",
            "nosa_dense_decode", "nosa_read_error", "nosa_strerror", "nosa_select_noalloc"]
-NOALLOC_SELECT_SCRATCH = 2 << 20
+NOALLOC_SELECT_SCRATCH = 1 << 20
 
 
 def build(force=False, verbose=False):

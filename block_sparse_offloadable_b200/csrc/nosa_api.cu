@@ -127,11 +127,8 @@ size_t ws_bytes_of(const nosa_config *c, int which) {
         const int n = select_nchunks(c, g);
         return n > 1 ? counters + (size_t)g.units * n * 32 * sizeof(uint64_t) : 0;
     }
-    if (which == NOSA_WS_SPARSE_DECODE || which == NOSA_WS_DENSE_DECODE) {
-        const int n = decode_chunks((int32_t)g.units,
-                                    (int32_t)(which == NOSA_WS_SPARSE_DECODE ? g.max_sel : g.nblk));
-        return n > 1 ? counters + (size_t)g.units * n * kPartFloats * sizeof(float) : 0;
-    }
+    if (which == NOSA_WS_SPARSE_DECODE || which == NOSA_WS_DENSE_DECODE)
+        return counters + (size_t)decode_ctas() * 2 * kPartFloats * sizeof(float);
     return 0;
 }
 
@@ -187,15 +184,9 @@ int run_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q, co
     p.max_sel = (int32_t)g.max_sel;
     p.G = (int32_t)g.G;
     p.units = (int32_t)g.units;
-    const int32_t max_blocks = (int32_t)(dense ? g.nblk : g.max_sel);
-    p.nchunks = decode_chunks(p.units, max_blocks);
-    p.max_nb = (max_blocks + p.nchunks - 1) / p.nchunks + 1;
     p.qk_log2 = c->scale * 1.4426950408889634f;
-    if (p.nchunks > 1) {
-        p.counter = static_cast<int32_t *>(ws);
-        p.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) +
-                                           align256((size_t)g.units * sizeof(int32_t)));
-    }
+    p.counter = static_cast<int32_t *>(ws);
+    p.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + align256((size_t)g.units * sizeof(int32_t)));
     return launch_decode(p, map, static_cast<cudaStream_t>(stream));
 }
 
@@ -216,6 +207,7 @@ int nosa_validate_config(const nosa_config *c) {
         return NOSA_ERR_UNSUPPORTED;
     if (c->max_ctx > kMaxCtx) return NOSA_ERR_CAPACITY;
     const int64_t units = (int64_t)c->batch * c->heads_kv;
+    if (units > kMaxUnits) return NOSA_ERR_CAPACITY;
     const int64_t rows = units * (c->max_ctx / kBlock) * 2 * kBlock;
     if (rows >= (1ll << 31)) return NOSA_ERR_CAPACITY;
     return NOSA_OK;

@@ -63,13 +63,12 @@ struct DecodeParams {
     const float *e;             // [u][max_ctx]
     const int32_t *seq_len;     // [u]
     uint16_t *out;              // [B][Hq][D]
-    float *part;                // [u][nchunks][kPartFloats]
+    float *part;                // [decode CTAs][2][kPartFloats]: first / last segment partials
     int32_t *counter;           // [u]
     uint32_t *err;
     int64_t max_ctx;
     int32_t blocks_per_unit;    // blocks per unit in the tensor-mapped buffer (nblk or nslots)
-    int32_t max_sel, G, units, nchunks;
-    int32_t max_nb;             // upper bound on blocks per CTA: ceil(max blocks / nchunks) + 1
+    int32_t max_sel, G, units;
     float qk_log2;              // scale * log2(e)
 };
 
@@ -82,7 +81,8 @@ int launch_decode(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t s
 
 // Launch geometry, shared by the launchers and the workspace-size queries.
 int select_chunk_blocks(int32_t units, int32_t nblk);
-int decode_chunks(int32_t units, int32_t max_blocks);
+int decode_ctas();
+constexpr int kMaxUnits = 2048;  // (seq, kv head) units per call: the decode kernel's prefix sums live in shared memory
 
 constexpr int kNumSms = 148;
 

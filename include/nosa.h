@@ -61,7 +61,8 @@ extern "C" {
  * Problem configuration.  Built: head_dim 128, block 64, sub_block 16,
  * local_blocks 1, 1 <= heads_q/heads_kv <= 8, 0 <= k_q <= 32,
  * 0 <= k_e <= 256, max_ctx a positive multiple of 64 and <= 2^20, and
- * batch * heads_kv * max_ctx * 2 < 2^31 (tensor-map row coordinates).
+ * batch * heads_kv <= 2048, and batch * heads_kv * max_ctx * 2 < 2^31
+ * (tensor-map row coordinates).
  */
 typedef struct nosa_config {
     int32_t batch;        /* B sequences */
@@ -271,7 +272,7 @@ int nosa_read_error(const nosa_state *st, uint32_t *flags, int clear, void *stre
  * one array, which keeps the last call's contents: calls that overlap on the
  * GPU (other streams, other threads) race and must not be issued.
  */
-#define NOSA_NOALLOC_SELECT_SCRATCH (2u << 20)
+#define NOSA_NOALLOC_SELECT_SCRATCH (1u << 20)
 int nosa_select_noalloc(const nosa_config *cfg, const nosa_state *st, const uint16_t *q,
                         int32_t *sel, int32_t *nsel, int32_t *gq, void *stream);
 

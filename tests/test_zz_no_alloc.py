@@ -44,9 +44,9 @@ def test_noalloc_select_matches_workspace_select(B, Hq, Hkv, k_q, k_e, L0):
 
 
 def test_noalloc_rejects_oversize_workspace():
-    # 8192 (sequence, kv head) units need more select scratch than the fixed array holds;
-    # the call is refused before anything is touched or launched
-    cfg = nosa.make_config(4096, 16, 2, 32, 32, 64000)
+    # 2048 (sequence, kv head) units at 128K context need more select scratch than the
+    # fixed array holds; the call is refused before anything is touched or launched
+    cfg = nosa.make_config(1024, 16, 2, 16, 48, 131072)
     assert nosa.nosa_validate_config(cfg) == nosa.OK
     assert nosa.nosa_workspace_bytes(cfg, nosa.WS_SELECT) > nosa.NOALLOC_SELECT_SCRATCH
     q = torch.zeros(16, dtype=torch.int16, device="cuda")
