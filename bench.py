@@ -56,24 +56,34 @@ def describe(c, groups):
 
 
 class Workload:
-    """All layers of one configuration: state, prefilled context and per-step inputs on the device."""
+    """All layers of one configuration: state, prefilled context and per-step inputs on the device.
 
-    def __init__(self, c, n_steps, seed=0, groups=2, layers=None, device="cuda"):
+    The batch is split into `micro` micro-batches of consecutive sequences, each with its own
+    per-layer state; micro-batch m runs its chain of layers on its own CUDA stream, so one
+    micro-batch's host->device fetch overlaps another's HBM-bound select and attention.  Every
+    sequence still goes through its layers in order.
+    """
+
+    def __init__(self, c, n_steps, seed=0, groups=2, layers=None, device="cuda", micro=1):
         self.c, self.seed, self.groups = c, seed, groups
         self.L = layers if layers is not None else c["layers"]
         self.B, self.Hq, self.Hkv = c["B"], c["Hq"], c["Hkv"]
+        assert self.B % micro == 0, "batch must split evenly into micro-batches"
+        self.micro, self.Bm = micro, self.B // micro
         self.units = self.B * self.Hkv
+        self.units_m = self.Bm * self.Hkv
         self.n_steps = n_steps
         self.max_ctx = (c["L"] + n_steps + 63) // 64 * 64
-        self.cfg = nosa.make_config(self.B, self.Hq, self.Hkv, c["k_q"], c["k_e"], self.max_ctx, c["offload"])
+        self.cfg = nosa.make_config(self.Bm, self.Hq, self.Hkv, c["k_q"], c["k_e"], self.max_ctx, c["offload"])
         dev = torch.device(device)
-        self.host = []
+        self.host = {}
         if c["offload"]:
             nbytes = nosa.nosa_state_bytes(self.cfg, nosa.BUF_KV_STORE)
-            self.host = [torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
-                         for _ in range(min(groups, self.L))]
-        self.layers = [nosa.NosaLayer(self.cfg, dev, self.host[l % len(self.host)] if self.host else None)
-                       for l in range(self.L)]
+            for g in range(min(groups, self.L)):
+                for m in range(micro):
+                    self.host[(g, m)] = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+        self.layers = [[nosa.NosaLayer(self.cfg, dev, self.host[(l % groups, m)] if self.host else None)
+                        for m in range(micro)] for l in range(self.L)]
         self._prefill(dev)
         self._inputs(dev)
 
@@ -83,85 +93,114 @@ class Workload:
 
     def _prefill(self, dev):
         T = self.c["L"]
-        k = torch.empty((self.units, T, D), dtype=torch.int16, device=dev)
+        k = torch.empty((self.units_m, T, D), dtype=torch.int16, device=dev)
         v = torch.empty_like(k)
-        e = torch.empty((self.units, T), dtype=torch.float32, device=dev)
-        for l, lay in enumerate(self.layers):
+        e = torch.empty((self.units_m, T), dtype=torch.float32, device=dev)
+        for l in range(self.L):
             kl = self.kv_layer(l)
-            synth.kv_dev(self.seed, synth.K_STREAM, kl, self.B, self.Hkv, 0, T, k)
-            synth.kv_dev(self.seed, synth.V_STREAM, kl, self.B, self.Hkv, 0, T, v)
-            synth.e_dev(self.seed, l, self.B, self.Hkv, 0, T, e)
-            lay.append(k, v, e, T)
+            for m, lay in enumerate(self.layers[l]):
+                s0 = m * self.Bm
+                synth.kv_dev(self.seed, synth.K_STREAM, kl, self.Bm, self.Hkv, 0, T, k, seq0=s0)
+                synth.kv_dev(self.seed, synth.V_STREAM, kl, self.Bm, self.Hkv, 0, T, v, seq0=s0)
+                synth.e_dev(self.seed, l, self.Bm, self.Hkv, 0, T, e, seq0=s0)
+                lay.append(k, v, e, T)
         torch.cuda.synchronize()
         del k, v, e
 
     def _inputs(self, dev):
-        """Per-step inputs of every layer, packed so one copy moves a step's inputs."""
-        n, U, L0 = self.n_steps, self.units, self.c["L"]
-        self.q_bytes = self.B * self.Hq * D * 2
-        self.kv_bytes = U * D * 2
-        self.e_bytes = U * 4
-        self.layer_in = self.q_bytes + 2 * self.kv_bytes + self.e_bytes
-        self.step_in = self.L * self.layer_in
+        """Per-step inputs of every layer and micro-batch, packed so one copy moves a step's inputs."""
+        n, Um, L0 = self.n_steps, self.units_m, self.c["L"]
+        self.q_bytes = self.Bm * self.Hq * D * 2
+        self.kv_bytes = Um * D * 2
+        self.e_bytes = Um * 4
+        self.part_in = self.q_bytes + 2 * self.kv_bytes + self.e_bytes
+        self.step_in = self.L * self.micro * self.part_in
         self.inputs = torch.empty((n, self.step_in), dtype=torch.uint8, device=dev)
-        qstate = torch.empty((self.B * self.Hq, D), dtype=torch.float32, device=dev)
-        qt = torch.empty((self.B * self.Hq, D), dtype=torch.int16, device=dev)
-        kk = torch.empty((U, n, D), dtype=torch.int16, device=dev)
+        qstate = torch.empty((self.Bm * self.Hq, D), dtype=torch.float32, device=dev)
+        qt = torch.empty((self.Bm * self.Hq, D), dtype=torch.int16, device=dev)
+        kk = torch.empty((Um, n, D), dtype=torch.int16, device=dev)
         vv = torch.empty_like(kk)
-        ee = torch.empty((U, n), dtype=torch.float32, device=dev)
+        ee = torch.empty((Um, n), dtype=torch.float32, device=dev)
         for l in range(self.L):
             kl = self.kv_layer(l)
-            synth.kv_dev(self.seed, synth.K_STREAM, kl, self.B, self.Hkv, L0, n, kk)
-            synth.kv_dev(self.seed, synth.V_STREAM, kl, self.B, self.Hkv, L0, n, vv)
-            synth.e_dev(self.seed, l, self.B, self.Hkv, L0, n, ee)
-            base = l * self.layer_in
-            for t in range(n):
-                synth.q_dev(self.seed, l, self.B, self.Hq, t, qstate, qt)
-                row = self.inputs[t]
-                row[base:base + self.q_bytes].view(torch.int16).copy_(qt.view(-1))
-                o = base + self.q_bytes
-                row[o:o + self.kv_bytes].view(torch.int16).copy_(kk[:, t].reshape(-1))
-                o += self.kv_bytes
-                row[o:o + self.kv_bytes].view(torch.int16).copy_(vv[:, t].reshape(-1))
-                o += self.kv_bytes
-                row[o:o + self.e_bytes].view(torch.float32).copy_(ee[:, t])
+            for m in range(self.micro):
+                s0 = m * self.Bm
+                synth.kv_dev(self.seed, synth.K_STREAM, kl, self.Bm, self.Hkv, L0, n, kk, seq0=s0)
+                synth.kv_dev(self.seed, synth.V_STREAM, kl, self.Bm, self.Hkv, L0, n, vv, seq0=s0)
+                synth.e_dev(self.seed, l, self.Bm, self.Hkv, L0, n, ee, seq0=s0)
+                base = (l * self.micro + m) * self.part_in
+                for t in range(n):
+                    synth.q_dev(self.seed, l, self.Bm, self.Hq, t, qstate, qt, seq0=s0)
+                    row = self.inputs[t]
+                    row[base:base + self.q_bytes].view(torch.int16).copy_(qt.view(-1))
+                    o = base + self.q_bytes
+                    row[o:o + self.kv_bytes].view(torch.int16).copy_(kk[:, t].reshape(-1))
+                    o += self.kv_bytes
+                    row[o:o + self.kv_bytes].view(torch.int16).copy_(vv[:, t].reshape(-1))
+                    o += self.kv_bytes
+                    row[o:o + self.e_bytes].view(torch.float32).copy_(ee[:, t])
         self.cur = torch.empty(self.step_in, dtype=torch.uint8, device=dev)
         self.out = torch.empty((self.L, self.B, self.Hq, D), dtype=torch.int16, device=dev)
+        self.streams = [torch.cuda.Stream(device=dev) for _ in range(self.micro - 1)]
         torch.cuda.synchronize()
 
-    def views(self, buf, l):
-        base = l * self.layer_in
-        q = buf[base:base + self.q_bytes].view(torch.int16).view(self.B, self.Hq, D)
+    def views(self, buf, l, m=0):
+        base = (l * self.micro + m) * self.part_in
+        q = buf[base:base + self.q_bytes].view(torch.int16).view(self.Bm, self.Hq, D)
         o = base + self.q_bytes
-        k = buf[o:o + self.kv_bytes].view(torch.int16).view(self.units, 1, D)
+        k = buf[o:o + self.kv_bytes].view(torch.int16).view(self.units_m, 1, D)
         o += self.kv_bytes
-        v = buf[o:o + self.kv_bytes].view(torch.int16).view(self.units, 1, D)
+        v = buf[o:o + self.kv_bytes].view(torch.int16).view(self.units_m, 1, D)
         o += self.kv_bytes
-        e = buf[o:o + self.e_bytes].view(torch.float32).view(self.units, 1)
+        e = buf[o:o + self.e_bytes].view(torch.float32).view(self.units_m, 1)
         return q, k, v, e
 
-    def launch_step(self, buf=None, events=None):
-        """Launch one decode step of every layer reading inputs from buf (default: self.cur)."""
+    def out_view(self, l, m):
+        return self.out[l, m * self.Bm:(m + 1) * self.Bm]
+
+    def kernel_calls(self, l, m, buf=None):
+        """(name, call) of one layer's step for micro-batch m, in order."""
         buf = self.cur if buf is None else buf
-        for l, lay in enumerate(self.layers):
-            q, k, v, e = self.views(buf, l)
-            parts = [("append", lambda: lay.append(k, v, e, 1)), ("select", lambda: lay.select(q))]
-            if self.c["offload"]:
-                parts.append(("cache_sync", lambda: lay.cache_sync()))
-            parts.append(("decode", lambda: lay.sparse_decode(q, self.out[l])))
-            for name, fn in parts:
-                if events is not None:
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record()
-                    fn()
-                    e1.record()
-                    events.append((name, l, e0, e1))
-                else:
-                    fn()
+        lay = self.layers[l][m]
+        q, k, v, e = self.views(buf, l, m)
+        out = self.out_view(l, m)
+        calls = [("append", lambda s: lay.append(k, v, e, 1, None, s)), ("select", lambda s: lay.select(q, s))]
+        if self.c["offload"]:
+            calls.append(("cache_sync", lambda s: lay.cache_sync(s)))
+        calls.append(("decode", lambda s: lay.sparse_decode(q, out, s)))
+        return calls
+
+    def launch_step(self, buf=None, events=None):
+        """Launch one decode step of every layer and micro-batch.
+
+        With events: everything on the current stream, each call bracketed by CUDA events (the
+        per-kernel timing pass).  Otherwise micro-batch m > 0 runs on its own stream, forked from
+        and joined back into the current stream."""
+        cur = torch.cuda.current_stream()
+        if events is not None:
+            for l in range(self.L):
+                for m in range(self.micro):
+                    for name, fn in self.kernel_calls(l, m, buf):
+                        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        e0.record()
+                        fn(cur)
+                        e1.record()
+                        events.append((name, l, e0, e1))
+            return
+        streams = [cur] + self.streams
+        for s in self.streams:
+            s.wait_stream(cur)
+        for l in range(self.L):
+            for m in range(self.micro):
+                for _, fn in self.kernel_calls(l, m, buf):
+                    fn(streams[m])
+        for s in self.streams:
+            cur.wait_stream(s)
 
     @property
     def launches_per_step(self):
-        return self.L * (4 if self.c["offload"] else 3)
+        # append, select, [cache plan, cache gather], decode
+        return self.L * self.micro * (5 if self.c["offload"] else 3)
 
 
 # ---------------------------------------------------------------------------------------
@@ -194,12 +233,14 @@ def time_idempotent(wl, name, reps, flush=None):
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
-        for l, lay in enumerate(wl.layers):
-            q, _, _, _ = wl.views(wl.cur, l)
-            if name == "select":
-                lay.select(q)
-            else:
-                lay.sparse_decode(q, wl.out[l])
+        for l in range(wl.L):
+            for m in range(wl.micro):
+                lay = wl.layers[l][m]
+                q, _, _, _ = wl.views(wl.cur, l, m)
+                if name == "select":
+                    lay.select(q)
+                else:
+                    lay.sparse_decode(q, wl.out_view(l, m))
     torch.cuda.synchronize()
     g.replay()
     torch.cuda.synchronize()
@@ -214,7 +255,7 @@ def time_idempotent(wl, name, reps, flush=None):
         torch.cuda.synchronize()
         total += e0.elapsed_time(e1)
     del g
-    return total / (reps * wl.L)
+    return total / (reps * wl.L * wl.micro)
 
 
 def measure_pcie_h2d(dev, nbytes=1 << 30):
@@ -357,7 +398,8 @@ def run_nosa(args, c, rank, world, dev):
     assert n_steps <= c["steps"] + 64, "more decode steps than the workload's context margin"
     t_setup = time.time()
     pcie = measure_pcie_h2d(dev) if c["offload"] else None
-    wl = Workload(c, n_steps, seed=args.seed, groups=args.host_groups, device=dev, layers=args.layers)
+    micro = args.micro if args.micro else (2 if c["offload"] else 1)
+    wl = Workload(c, n_steps, seed=args.seed, groups=args.host_groups, device=dev, layers=args.layers, micro=micro)
     setup_s = time.time() - t_setup
     stream = torch.cuda.current_stream()
     step_i = 0
@@ -435,9 +477,10 @@ def run_nosa(args, c, rank, world, dev):
         wl.launch_step(events=events)
         step_i += 1
         torch.cuda.synchronize()
+        all_layers = [lay for per_layer in wl.layers for lay in per_layer]
         if c["offload"]:
-            fetched.append(sum(int(lay.n_fetched.sum()) for lay in wl.layers))
-        for lay in wl.layers:
+            fetched.append(sum(int(lay.n_fetched.sum()) for lay in all_layers))
+        for lay in all_layers:
             nsel_sum += int(lay.nsel.sum())
             nsel_n += lay.units
     kt = {}
@@ -449,11 +492,11 @@ def run_nosa(args, c, rank, world, dev):
         kt[name] = [per] * len(kt[name])
     nsel_mean = nsel_sum / max(nsel_n, 1)
     hbm_peak, peak_kind = load_peaks()
-    U, Lctx = wl.units, c["L"] + step_i
+    U, Lctx = wl.units_m, c["L"] + step_i
     nb_c = (Lctx - 1) // 64
-    algo = {  # algorithmic bytes per launch (per layer)
+    algo = {  # algorithmic bytes per launch (one layer of one micro-batch)
         "select": U * (nb_c * 4 * D * 4 + (c["Hq"] // c["Hkv"]) * D * 2),
-        "decode": U * nsel_mean * (64 * D * 2 * 2 + 64 * 4) + 2 * c["B"] * c["Hq"] * D * 2,
+        "decode": U * nsel_mean * (64 * D * 2 * 2 + 64 * 4) + 2 * wl.Bm * c["Hq"] * D * 2,
         "append": U * (2 * D * 2 + 4),
     }
     kern = {}
@@ -465,7 +508,7 @@ def run_nosa(args, c, rank, world, dev):
             kern[name].update({"bytes": algo[name], "GBps": gbs, "frac_hbm": gbs / hbm_peak})
     pcie_obj = None
     if c["offload"] and fetched:
-        fb = sum(fetched) / len(fetched) / wl.L  # blocks per layer-step
+        fb = sum(fetched) / len(fetched) / (wl.L * wl.micro)  # blocks per launch (layer, micro-batch)
         avg = sum(kt["cache_sync"]) / len(kt["cache_sync"])
         gbs = fb * 32768 / (avg * 1e-3) / 1e9
         kern["cache_sync"].update({"bytes": fb * 32768, "GBps": gbs, "frac_pcie": gbs / pcie})
@@ -474,7 +517,7 @@ def run_nosa(args, c, rank, world, dev):
                     "peak": "measured pinned cudaMemcpyAsync H2D, 1 GiB, this box", "frac": gbs / pcie}
     dom = max(kern, key=lambda k: kern[k]["share"])
     if dom == "cache_sync" and pcie_obj:
-        roof = {"bound": "pcie", "kernel": "cache_sync (K3+K4 gather)", "achieved": pcie_obj["achieved_GBps"],
+        roof = {"bound": "pcie", "kernel": "cache_sync (plan + gather)", "achieved": pcie_obj["achieved_GBps"],
                 "peak": pcie, "unit": "GB/s", "frac": pcie_obj["frac"], "traffic": None,
                 "peak_source": "measured live: pinned H2D copy"}
     else:
@@ -510,7 +553,7 @@ def run_nosa(args, c, rank, world, dev):
                "path": "pinned host inputs -> nosa_* C ABI -> pinned host outputs"}
         step_i += k_e2e
 
-    errs = [lay.read_error() for lay in wl.layers]
+    errs = [lay.read_error() for per_layer in wl.layers for lay in per_layer]
     if any(errs):
         raise RuntimeError(f"device error flags set: {errs}")
     cpu = None
@@ -528,7 +571,7 @@ def run_nosa(args, c, rank, world, dev):
         "config": {"workload": f"config {args.config}: " + describe(c, args.host_groups), "layers": c["layers"],
                    "batch": c["B"], "heads_q": c["Hq"], "heads_kv": c["Hkv"], "context": c["L"], "k_q": c["k_q"],
                    "k_e": c["k_e"], "offload": c["offload"], "host_kv_groups": args.host_groups if c["offload"] else None,
-                   "cuda_graph": graph is not None,
+                   "cuda_graph": graph is not None, "micro_batches": wl.micro,
                    "l2": ("L2 flushed (256 MB write) before every timed step; steps timed one by one" if small else
                           f"inputs larger than L2: each step streams {step_bytes(wl) / 1e9:.2f} GB of pooled keys and KV blocks"),
                    "kernel_timing": "select/decode: CUDA graph of all layers replayed; append/cache_sync: events per launch"},
@@ -550,6 +593,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--host-groups", type=int, default=2)
     ap.add_argument("--layers", type=int, default=None, help="override the layer count (profiling captures)")
+    ap.add_argument("--micro", type=int, default=0,
+                    help="micro-batches on separate streams (default: 2 with offload, else 1)")
     ap.add_argument("--profile-steps", type=int, default=3)
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

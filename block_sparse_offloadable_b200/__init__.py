@@ -28,7 +28,7 @@ OK, ERR_ARG, ERR_CAPACITY, ERR_PTR, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED, ERR_
 EFLAG_CAPACITY, EFLAG_TIMEOUT, EFLAG_NOSLOT, EFLAG_STATE = 1, 2, 4, 8
 (BUF_KV_STORE, BUF_EVICT_LOGIT, BUF_CK, BUF_BLK_EVICT, BUF_GAMMA_E, BUF_GAMMA_N, BUF_SEQ_LEN, BUF_CACHE,
  BUF_SLOT_BLOCK, BUF_BLOCK_SLOT, BUF_ERR) = range(11)
-WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE = 0, 1, 2
+WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC = 0, 1, 2, 3
 
 # Every extern "C" symbol include/nosa.h declares.
 EXPORTS = ["nosa_validate_config", "nosa_state_bytes", "nosa_workspace_bytes", "nosa_state_init",
@@ -84,7 +84,7 @@ def lib():
         L.nosa_state_init.argtypes = [C, S, P]
         L.nosa_compress_append.argtypes = [C, S, P, P, P, ctypes.c_int32, P, P]
         L.nosa_select.argtypes = [C, S, P, P, P, P, P, ctypes.c_size_t, P]
-        L.nosa_cache_sync.argtypes = [C, S, P, P, P, P, P]
+        L.nosa_cache_sync.argtypes = [C, S, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_sparse_decode.argtypes = [C, S, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_dense_decode.argtypes = [C, S, P, P, P, ctypes.c_size_t, P]
         L.nosa_read_error.argtypes = [S, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P]
@@ -157,9 +157,10 @@ def nosa_select_noalloc(cfg, st, q, sel, nsel, gq=None, stream=None):
                                      _stream(stream)), "nosa_select_noalloc")
 
 
-def nosa_cache_sync(cfg, st, sel, nsel, block_table, n_fetched=None, stream=None):
+def nosa_cache_sync(cfg, st, sel, nsel, block_table, n_fetched=None, ws=None, stream=None):
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib().nosa_cache_sync(ctypes.byref(cfg), ctypes.byref(st), _ptr(sel), _ptr(nsel), _ptr(block_table),
-                                 _ptr(n_fetched), _stream(stream)), "nosa_cache_sync")
+                                 _ptr(n_fetched), _ptr(ws), nbytes, _stream(stream)), "nosa_cache_sync")
 
 
 def nosa_sparse_decode(cfg, st, q, sel, nsel, block_table, out, ws=None, stream=None):
@@ -243,6 +244,7 @@ class NosaLayer:
         self.ws_select = ws(WS_SELECT)
         self.ws_decode = ws(WS_SPARSE_DECODE)
         self.ws_dense = None if cfg.offload else ws(WS_DENSE_DECODE)
+        self.ws_cache = ws(WS_CACHE_SYNC)
         nosa_state_init(cfg, self.state)
 
     # one decode step = the four calls, in order
@@ -253,7 +255,8 @@ class NosaLayer:
         nosa_select(self.cfg, self.state, q, self.sel, self.nsel, self.gq, self.ws_select, stream)
 
     def cache_sync(self, stream=None):
-        nosa_cache_sync(self.cfg, self.state, self.sel, self.nsel, self.block_table, self.n_fetched, stream)
+        nosa_cache_sync(self.cfg, self.state, self.sel, self.nsel, self.block_table, self.n_fetched, self.ws_cache,
+                        stream)
 
     def sparse_decode(self, q, out, stream=None):
         bt = self.block_table if self.cfg.offload else None

@@ -129,6 +129,8 @@ size_t ws_bytes_of(const nosa_config *c, int which) {
     }
     if (which == NOSA_WS_SPARSE_DECODE || which == NOSA_WS_DENSE_DECODE)
         return counters + (size_t)decode_ctas() * 2 * kPartFloats * sizeof(float);
+    if (which == NOSA_WS_CACHE_SYNC)
+        return c->offload ? counters + (size_t)g.units * g.max_sel * sizeof(uint32_t) : 0;
     return 0;
 }
 
@@ -314,7 +316,8 @@ int nosa_select(const nosa_config *c, const nosa_state *st, const uint16_t *q, i
 }
 
 int nosa_cache_sync(const nosa_config *c, const nosa_state *st, const int32_t *sel,
-                    const int32_t *nsel, int32_t *block_table, int32_t *n_fetched, void *stream) {
+                    const int32_t *nsel, int32_t *block_table, int32_t *n_fetched, void *ws,
+                    size_t ws_bytes, void *stream) {
     Geo g;
     int rc;
     if ((rc = nosa_validate_config(c))) return rc;
@@ -325,6 +328,7 @@ int nosa_cache_sync(const nosa_config *c, const nosa_state *st, const int32_t *s
         (rc = check_dev(block_table, false)))
         return rc;
     if (n_fetched && (rc = check_dev(n_fetched, false))) return rc;
+    if ((rc = check_ws(c, NOSA_WS_CACHE_SYNC, ws, ws_bytes))) return rc;
     uint8_t *s;
     if ((rc = store_addr(c, st, &s))) return rc;
     CacheParams p;
@@ -332,6 +336,9 @@ int nosa_cache_sync(const nosa_config *c, const nosa_state *st, const int32_t *s
     p.sel = sel; p.nsel = nsel; p.store = s; p.cache = static_cast<uint8_t *>(st->cache);
     p.slot_block = st->slot_block; p.block_slot = st->block_slot; p.block_table = block_table;
     p.n_fetched = n_fetched; p.err = st->err;
+    p.miss_count = static_cast<int32_t *>(ws);
+    p.miss_list = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) +
+                                               align256((size_t)g.units * sizeof(int32_t)));
     p.nblk = (int32_t)g.nblk; p.nslots = (int32_t)g.nslots; p.units = (int32_t)g.units;
     p.max_sel = (int32_t)g.max_sel;
     return launch_cache_sync(p, static_cast<cudaStream_t>(stream));

@@ -50,7 +50,9 @@ struct CacheParams {
     int32_t *slot_block;      // [u][nslots]
     int32_t *block_slot;      // [u][nblk]
     int32_t *block_table;     // [u][max_sel]
-    int32_t *n_fetched;       // [u] or null
+    int32_t *n_fetched;       // [u] or null: copy of miss_count
+    int32_t *miss_count;      // [u] workspace: blocks to fetch per unit
+    uint32_t *miss_list;      // [u][max_sel] workspace: (slot << 20 | block) of each block to fetch
     uint32_t *err;
     int32_t nblk, nslots, units, max_sel;
 };

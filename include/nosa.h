@@ -127,7 +127,12 @@ enum nosa_buffer {
     NOSA_BUF_COUNT
 };
 
-enum nosa_call { NOSA_WS_SELECT = 0, NOSA_WS_SPARSE_DECODE = 1, NOSA_WS_DENSE_DECODE = 2 };
+enum nosa_call {
+    NOSA_WS_SELECT = 0,
+    NOSA_WS_SPARSE_DECODE = 1,
+    NOSA_WS_DENSE_DECODE = 2,
+    NOSA_WS_CACHE_SYNC = 3
+};
 
 /* Validate a configuration: NOSA_OK or a negative code. */
 int nosa_validate_config(const nosa_config *cfg);
@@ -208,15 +213,18 @@ int nosa_select(const nosa_config *cfg, const nosa_state *st, const uint16_t *q,
  *   sel, nsel    from nosa_select
  *   block_table  device int32 [u][k_q+k_e+1] out: cache slot of each sel entry, -1 padded
  *   n_fetched    device int32 [u] out or NULL: blocks fetched from the host this step
+ *   ws           device workspace of nosa_workspace_bytes(cfg, NOSA_WS_CACHE_SYNC) bytes
  *
  * Frees every slot whose block is not in S(t), assigns the freed slots (in
  * ascending order) to the blocks of S(t) that are not resident (in ascending
  * block order), and copies each such block (32 KiB: keys and values) from the
  * host store into its slot with 16-byte loads through the device mapping of
- * host memory.  Offload mode only (NOSA_ERR_ARG otherwise).
+ * host memory, the copy split evenly over all SMs.  Offload mode only
+ * (NOSA_ERR_ARG otherwise).
  */
 int nosa_cache_sync(const nosa_config *cfg, const nosa_state *st, const int32_t *sel,
-                    const int32_t *nsel, int32_t *block_table, int32_t *n_fetched, void *stream);
+                    const int32_t *nsel, int32_t *block_table, int32_t *n_fetched, void *ws,
+                    size_t ws_bytes, void *stream);
 
 /*
  * a5 -- sparse decode.  NOSA pages: gist.science "ED-DMA" (the exponent of

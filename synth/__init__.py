@@ -55,9 +55,9 @@ def gpu():
         build(gpu=True)
         L = ctypes.CDLL(_GPU_SO)
         u64, u32, i64, i32, P = ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p
-        L.nosa_synth_kv_dev.argtypes = [u64, u32, u32, i32, i32, u64, i64, i32, P, P]
-        L.nosa_synth_e_dev.argtypes = [u64, u32, i32, i32, u64, i64, P, P]
-        L.nosa_synth_q_dev.argtypes = [u64, u32, i32, i32, i64, i32, P, P, P]
+        L.nosa_synth_kv_dev.argtypes = [u64, u32, u32, i32, i32, i32, u64, i64, i32, P, P]
+        L.nosa_synth_e_dev.argtypes = [u64, u32, i32, i32, i32, u64, i64, P, P]
+        L.nosa_synth_q_dev.argtypes = [u64, u32, i32, i32, i32, i64, i32, P, P, P]
         _gpu = L
     return _gpu
 
@@ -98,15 +98,17 @@ def _check(rc, what):
         raise RuntimeError(f"synth {what} failed ({rc})")
 
 
-def kv_dev(seed, stream, layer, B, Hkv, p0, T, out, cuda_stream=0, D=128):
-    """Fill out ([B*Hkv][T][D] bf16, device) with K or V rows of positions p0..p0+T-1."""
-    _check(gpu().nosa_synth_kv_dev(seed, stream, layer, B, Hkv, p0, T, D, out.data_ptr(), cuda_stream), "kv")
+def kv_dev(seed, stream, layer, B, Hkv, p0, T, out, cuda_stream=0, D=128, seq0=0):
+    """Fill out ([B*Hkv][T][D] bf16, device) with K or V rows of sequences seq0..seq0+B-1,
+    positions p0..p0+T-1."""
+    _check(gpu().nosa_synth_kv_dev(seed, stream, layer, seq0, B, Hkv, p0, T, D, out.data_ptr(), cuda_stream), "kv")
 
 
-def e_dev(seed, layer, B, Hkv, p0, T, out, cuda_stream=0):
-    _check(gpu().nosa_synth_e_dev(seed, layer, B, Hkv, p0, T, out.data_ptr(), cuda_stream), "e")
+def e_dev(seed, layer, B, Hkv, p0, T, out, cuda_stream=0, seq0=0):
+    _check(gpu().nosa_synth_e_dev(seed, layer, seq0, B, Hkv, p0, T, out.data_ptr(), cuda_stream), "e")
 
 
-def q_dev(seed, layer, B, Hq, t, state, out, cuda_stream=0, D=128):
+def q_dev(seed, layer, B, Hq, t, state, out, cuda_stream=0, D=128, seq0=0):
     """Advance the fp32 query state [B*Hq][D] to step t and write bf16 queries into out."""
-    _check(gpu().nosa_synth_q_dev(seed, layer, B, Hq, t, D, state.data_ptr(), out.data_ptr(), cuda_stream), "q")
+    _check(gpu().nosa_synth_q_dev(seed, layer, seq0, B, Hq, t, D, state.data_ptr(), out.data_ptr(), cuda_stream),
+           "q")
