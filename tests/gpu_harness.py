@@ -109,13 +109,59 @@ def _tie_ok(sa, sb, smax):
     return abs(sa - sb) <= TIE_REL * max(abs(sa), abs(sb), 1e-6 * smax)
 
 
+def new_stats():
+    return dict(cmp=0, exact=0, excused=0, unexcused=0, ge_mismatch=0, fetch_cmp=0, fetch_mismatch=0,
+                max_abs=0.0, sum_abs=0.0, n_out=0, max_rel=0.0, dense_max_abs=0.0, dense_max_rel=0.0,
+                gamma_min=1.0)
+
+
+def compare_step(st, o, r, q, gsel, ggq, gge, gout, k_q, history_ok, gfetch=None, report=None, tag=None):
+    """Compare one (unit, step) of the GPU path with the oracle's step result r.
+
+    gsel: GPU S(t) (ascending, local last); ggq: GPU Gamma_q ids (rank order, -1 padded);
+    gge: GPU Gamma_e ids (any order) or None; gout: GPU output [G][D] as float.
+    Returns the updated history flag (False once the selections have differed)."""
+    st["cmp"] += 1
+    if gge is not None and not np.array_equal(np.sort(gge), r["ge"]):
+        st["ge_mismatch"] += 1
+    if np.array_equal(gsel, r["sel"]):
+        st["exact"] += 1
+        ref = r["o"]
+    else:
+        history_ok = False
+        gq_set = set(x for x in list(ggq)[:k_q] if x >= 0)
+        oq_set = set(r["gq"].tolist())
+        s = r["scores"]
+        smax = float(np.abs(s).max()) if len(s) else 0.0
+        a = sorted(gq_set - oq_set, key=lambda x: -s[x])
+        bb = sorted(oq_set - gq_set, key=lambda x: -s[x])
+        consistent = np.array_equal(gsel, np.array(sorted(gq_set | set(r["ge"].tolist())) + [r["local"]]))
+        if consistent and len(a) == len(bb) and all(_tie_ok(s[x], s[y], smax) for x, y in zip(a, bb)):
+            st["excused"] += 1
+        else:
+            st["unexcused"] += 1
+            if report is not None:
+                report.append((tag, list(gsel), r["sel"].tolist()))
+        ref = o.attend_blocks(q, gsel)
+    err = np.abs(gout - ref)
+    st["max_abs"] = max(st["max_abs"], float(err.max()))
+    st["sum_abs"] += float(err.sum())
+    st["n_out"] += err.size
+    st["max_rel"] = max(st["max_rel"], float(np.linalg.norm(gout - ref) / max(np.linalg.norm(ref), 1e-30)))
+    if r["gamma"] >= 0:
+        st["gamma_min"] = min(st["gamma_min"], r["gamma"])
+    if gfetch is not None and history_ok:
+        st["fetch_cmp"] += 1
+        if int(gfetch) != r["n_fetch"]:
+            st["fetch_mismatch"] += 1
+    return history_ok
+
+
 def compare(sc, data, gpu, units=None, report=None):
     """Compare every (step, unit) of `units` against the oracle; returns a stats dict."""
     K, V, E, Q = data
     units = range(sc.units) if units is None else units
-    st = dict(cmp=0, exact=0, excused=0, unexcused=0, ge_mismatch=0, fetch_cmp=0, fetch_mismatch=0,
-              max_abs=0.0, sum_abs=0.0, n_out=0, max_rel=0.0, dense_max_abs=0.0, dense_max_rel=0.0,
-              gamma_min=1.0)
+    st = new_stats()
     for u in units:
         b, g = divmod(u, sc.Hkv)
         n0 = sc.lens[b]
@@ -128,42 +174,10 @@ def compare(sc, data, gpu, units=None, report=None):
             q = Q[t, b, g * sc.G:(g + 1) * sc.G]
             r = o.step(K[u, p], V[u, p], float(E[u, p]), q)
             gsel = gpu["sel"][t][u][: gpu["nsel"][t][u]]
-            st["cmp"] += 1
-            if sc.k_e:
-                gge = np.sort(gpu["ge"][t][u][: gpu["gn"][t][u]])
-                if not np.array_equal(gge, r["ge"]):
-                    st["ge_mismatch"] += 1
-            if np.array_equal(gsel, r["sel"]):
-                st["exact"] += 1
-                ref = r["o"]
-            else:
-                history_ok = False
-                ggq = set(x for x in gpu["gq"][t][u][: sc.k_q].tolist() if x >= 0)
-                ogq = set(r["gq"].tolist())
-                s = r["scores"]
-                smax = float(np.abs(s).max()) if len(s) else 0.0
-                a = sorted(ggq - ogq, key=lambda x: -s[x])
-                bb = sorted(ogq - ggq, key=lambda x: -s[x])
-                consistent = np.array_equal(gsel, np.array(sorted(ggq | set(r["ge"].tolist())) + [r["local"]]))
-                if consistent and len(a) == len(bb) and all(_tie_ok(s[x], s[y], smax) for x, y in zip(a, bb)):
-                    st["excused"] += 1
-                else:
-                    st["unexcused"] += 1
-                    if report is not None:
-                        report.append((t, u, gsel.tolist(), r["sel"].tolist()))
-                ref = o.attend_blocks(q, gsel)
-            got = gpu["out"][t][b, g * sc.G:(g + 1) * sc.G]
-            err = np.abs(got - ref)
-            st["max_abs"] = max(st["max_abs"], float(err.max()))
-            st["sum_abs"] += float(err.sum())
-            st["n_out"] += err.size
-            st["max_rel"] = max(st["max_rel"], float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)))
-            if r["gamma"] >= 0:
-                st["gamma_min"] = min(st["gamma_min"], r["gamma"])
-            if sc.offload and history_ok:
-                st["fetch_cmp"] += 1
-                if int(gpu["nf"][t][u]) != r["n_fetch"]:
-                    st["fetch_mismatch"] += 1
+            gge = gpu["ge"][t][u][: gpu["gn"][t][u]] if sc.k_e else None
+            history_ok = compare_step(st, o, r, q, gsel, gpu["gq"][t][u], gge,
+                                      gpu["out"][t][b, g * sc.G:(g + 1) * sc.G], sc.k_q, history_ok,
+                                      gpu["nf"][t][u] if sc.offload else None, report, (t, u))
             if sc.dense:
                 dref = o.dense(q)
                 dg = gpu["dense"][t][b, g * sc.G:(g + 1) * sc.G]
