@@ -64,8 +64,8 @@ class Workload:
     sequence still goes through its layers in order.
     """
 
-    def __init__(self, c, n_steps, seed=0, groups=2, layers=None, device="cuda", micro=1):
-        self.c, self.seed, self.groups = c, seed, groups
+    def __init__(self, c, n_steps, seed=0, groups=2, layers=None, device="cuda", micro=1, seq_base=0):
+        self.c, self.seed, self.groups, self.seq_base = c, seed, groups, seq_base
         self.L = layers if layers is not None else c["layers"]
         self.B, self.Hq, self.Hkv = c["B"], c["Hq"], c["Hkv"]
         assert self.B % micro == 0, "batch must split evenly into micro-batches"
@@ -99,7 +99,7 @@ class Workload:
         for l in range(self.L):
             kl = self.kv_layer(l)
             for m, lay in enumerate(self.layers[l]):
-                s0 = m * self.Bm
+                s0 = self.seq_base + m * self.Bm
                 synth.kv_dev(self.seed, synth.K_STREAM, kl, self.Bm, self.Hkv, 0, T, k, seq0=s0)
                 synth.kv_dev(self.seed, synth.V_STREAM, kl, self.Bm, self.Hkv, 0, T, v, seq0=s0)
                 synth.e_dev(self.seed, l, self.Bm, self.Hkv, 0, T, e, seq0=s0)
@@ -124,7 +124,7 @@ class Workload:
         for l in range(self.L):
             kl = self.kv_layer(l)
             for m in range(self.micro):
-                s0 = m * self.Bm
+                s0 = self.seq_base + m * self.Bm
                 synth.kv_dev(self.seed, synth.K_STREAM, kl, self.Bm, self.Hkv, L0, n, kk, seq0=s0)
                 synth.kv_dev(self.seed, synth.V_STREAM, kl, self.Bm, self.Hkv, L0, n, vv, seq0=s0)
                 synth.e_dev(self.seed, l, self.Bm, self.Hkv, L0, n, ee, seq0=s0)
@@ -322,6 +322,20 @@ def gpu_index(local_rank):
     return local_rank
 
 
+def reduce_max_ms(ms, world, device):
+    """Device time of the slowest rank (every rank takes part; world 1 returns ms)."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(world, batch, steps, ms):
+    """Whole-job tokens/s: every rank decodes `batch` sequences per step; time = slowest rank."""
+    return world * batch * steps / (ms * 1e-3)
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -399,7 +413,9 @@ def run_nosa(args, c, rank, world, dev):
     t_setup = time.time()
     pcie = measure_pcie_h2d(dev) if c["offload"] else None
     micro = args.micro if args.micro else (2 if c["offload"] else 1)
-    wl = Workload(c, n_steps, seed=args.seed, groups=args.host_groups, device=dev, layers=args.layers, micro=micro)
+    # replicas: rank r decodes its own sequences r*B .. (r+1)*B-1 (no exchange between sequences)
+    wl = Workload(c, n_steps, seed=args.seed, groups=args.host_groups, device=dev, layers=args.layers, micro=micro,
+                  seq_base=rank * c["B"])
     setup_s = time.time() - t_setup
     stream = torch.cuda.current_stream()
     step_i = 0
@@ -459,11 +475,8 @@ def run_nosa(args, c, rank, world, dev):
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1)
     clk = clocks.stop()
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
-    value = world * c["B"] * args.steps / (ms * 1e-3)
+    ms = reduce_max_ms(ms, world, dev)
+    value = aggregate_value(world, c["B"], args.steps, ms)
     launches = wl.launches_per_step * args.steps
 
     # ---- per-kernel durations (events around every launch, eager) + selection stats ----
