@@ -3,12 +3,12 @@
 A step is one decode step of the whole stack: for every layer, append the new
 token of every sequence (nosa_compress_append), select (nosa_select), sync the
 block cache (nosa_cache_sync, offload mode) and attend (nosa_sparse_decode).
-Throughput = sequences x steps / device time.  Default workload (--config 4):
+Throughput = sequences x steps / device time.  Default workload (offload28-128k):
 28 layers, batch 64, 16 q / 2 kv heads, head_dim 128, 128K context, KV in
 pinned host memory with a device cache of local + 64 blocks per (seq, kv head),
 k_e = 48, k_q = 16.
 
-    python bench.py [--config 4] [--steps K] [--warmup W] [--gpus N] [--impl nosa|reference]
+    python bench.py [--workload offload28-128k] [--steps K] [--warmup W] [--gpus N] [--impl nosa|reference]
 
 --impl reference times the CPU oracle (the plain fp64 restatement of the
 method, single thread) on a bounded sample of the same workload.
@@ -36,12 +36,17 @@ import synth  # noqa: E402
 METRIC = "sparse decode tokens/s/GPU at 128K ctx; % of HBM and PCIe roofline"
 D = 128
 
-CONFIGS = {
-    1: dict(layers=1, B=1, Hq=16, Hkv=16, L=8192, k_q=16, k_e=48, steps=32, offload=False),
-    2: dict(layers=1, B=8, Hq=16, Hkv=2, L=16384, k_q=16, k_e=48, steps=128, offload=False),
-    3: dict(layers=28, B=32, Hq=16, Hkv=2, L=32768, k_q=16, k_e=48, steps=64, offload=False),
-    4: dict(layers=28, B=64, Hq=16, Hkv=2, L=131072, k_q=16, k_e=48, steps=256, offload=True),
+WORKLOADS = {
+    # one layer, batch 1, 16 q / 16 kv heads, 8K context, 32 decode steps, KV in device memory
+    "mha-8k": dict(layers=1, B=1, Hq=16, Hkv=16, L=8192, k_q=16, k_e=48, steps=32, offload=False),
+    # one layer, batch 8, GQA 16 q / 2 kv heads, 16K context, 128 decode steps, KV in device memory
+    "gqa-16k": dict(layers=1, B=8, Hq=16, Hkv=2, L=16384, k_q=16, k_e=48, steps=128, offload=False),
+    # 28-layer stack, batch 32, GQA 16/2, 32K context, 64 decode steps, KV in device memory
+    "stack28-32k": dict(layers=28, B=32, Hq=16, Hkv=2, L=32768, k_q=16, k_e=48, steps=64, offload=False),
+    # 28-layer stack, batch 64, GQA 16/2, 128K context, 256 decode steps, KV in pinned host memory
+    "offload28-128k": dict(layers=28, B=64, Hq=16, Hkv=2, L=131072, k_q=16, k_e=48, steps=256, offload=True),
 }
+DEFAULT_WORKLOAD = "offload28-128k"
 
 
 def describe(c, groups):
@@ -400,7 +405,7 @@ def run_reference(args, c, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"config {args.config}: " + describe(c, args.host_groups)},
+            "config": {"workload": f"{args.workload}: " + describe(c, args.host_groups)},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -581,7 +586,7 @@ def run_nosa(args, c, rank, world, dev):
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded counter-based generator: K,V ~ N(0,1)/sqrt(128) bf16, e ~ N(0,1), drifting q)",
-        "config": {"workload": f"config {args.config}: " + describe(c, args.host_groups), "layers": c["layers"],
+        "config": {"workload": f"{args.workload}: " + describe(c, args.host_groups), "layers": c["layers"],
                    "batch": c["B"], "heads_q": c["Hq"], "heads_kv": c["Hkv"], "context": c["L"], "k_q": c["k_q"],
                    "k_e": c["k_e"], "offload": c["offload"], "host_kv_groups": args.host_groups if c["offload"] else None,
                    "cuda_graph": graph is not None, "micro_batches": wl.micro,
@@ -601,7 +606,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=4, choices=sorted(CONFIGS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="nosa", choices=["nosa", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--host-groups", type=int, default=2)
@@ -613,7 +618,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    c = dict(CONFIGS[args.config])
+    c = dict(WORKLOADS[args.workload])
     if args.layers is not None:
         c["layers"] = args.layers
     world = int(os.environ.get("WORLD_SIZE", "1"))

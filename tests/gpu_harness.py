@@ -1,5 +1,5 @@
 """Run the CUDA path (through the C ABI) and the CPU oracle on the same seeded
-inputs, and compare them the way the benchmark spec's tolerances say:
+inputs, and compare them with the tolerances the library is held to:
 
 * selected block sets bit-exact, except near-ties: a differing pair of blocks
   whose oracle scores satisfy |s_a - s_b| <= 1e-4 * max(|s_a|, |s_b|, 1e-6 * max|s|)

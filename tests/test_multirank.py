@@ -61,7 +61,7 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     monkeypatch.setattr(bench, "oracle_sample", lambda *a, **k: called.append(1) or (1.0, 1, "x"))
 
     class Args:
-        host_groups, seed, warmup, steps, gpus, config = 2, 0, 1, 1, 2, 4
+        host_groups, seed, warmup, steps, gpus, workload = 2, 0, 1, 1, 2, "offload28-128k"
 
-    bench.run_reference(Args, dict(bench.CONFIGS[4]), rank=1)
+    bench.run_reference(Args, dict(bench.WORKLOADS["offload28-128k"]), rank=1)
     assert called == []
