@@ -201,6 +201,28 @@ __device__ __forceinline__ void list_offer(uint64_t &list, uint64_t cand, int la
     }
 }
 
+__device__ __forceinline__ uint64_t shfl_xor64(uint64_t v, int m) {
+    uint32_t lo = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(v), m);
+    uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(v >> 32), m);
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// Merge another warp-wide sorted list (descending, lane i = rank i) into `list`,
+// keeping the 32 best of both: the elementwise max of one list and the other
+// reversed is a bitonic sequence holding the top 32 of the union; five
+// half-cleaner stages sort it back into descending order.
+__device__ __forceinline__ void list_merge(uint64_t &list, uint64_t other, int lane) {
+    const uint64_t rev = shfl64(other, 31 - lane);
+    uint64_t m = list > rev ? list : rev;
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) {
+        const uint64_t p = shfl_xor64(m, j);
+        const bool lower = (lane & j) == 0;
+        m = lower ? (m > p ? m : p) : (m < p ? m : p);
+    }
+    list = m;
+}
+
 __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bits) {
     if (err) atomicOr(err, bits);
 }

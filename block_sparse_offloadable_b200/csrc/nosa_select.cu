@@ -55,12 +55,12 @@ size_t select_smem_bytes(int32_t nblk) {
 }  // namespace
 
 int select_chunk_blocks(int32_t units, int32_t nblk) {
-    // candidates per unit are at most nblk - 1; per-CTA fixed cost ~ 16 blocks
-    // (pipeline fill and the list merge)
+    // candidates per unit are at most nblk - 1; per-CTA fixed cost ~ 32 blocks
+    // (pipeline fill, the list merges, the atomic hand-off)
     const int64_t work = nblk > 1 ? nblk - 1 : 1;
     int64_t nmax = (work + kSelSB - 1) / kSelSB;
     if (nmax > kMaxChunks) nmax = kMaxChunks;
-    const int n = best_chunks(units, work, (int64_t)kNumSms * kCtasPerSm, 16, nmax);
+    const int n = best_chunks(units, work, (int64_t)kNumSms * kCtasPerSm, 32, nmax);
     int64_t per = (work + n - 1) / n;
     per = (per + kSelSB - 1) / kSelSB * kSelSB;
     return (int)per;
@@ -91,6 +91,18 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
         fence_mbar_init();
     }
     __syncthreads();
+
+    // warp 0 may finalize this unit: fetch Gamma_e now, while the stream runs
+    const int32_t ne = (warp == 0) ? min(p.gamma_n[u], p.k_e) : 0;
+    int32_t ge_reg[kMaxKe / 32];
+    if (warp == 0) {
+        const int32_t *ge = p.gamma_e + (int64_t)u * p.k_e;
+#pragma unroll
+        for (int i = 0; i < kMaxKe / 32; ++i) {
+            const int j = lane + 32 * i;
+            ge_reg[i] = (j < ne) ? ge[j] : -1;
+        }
+    }
 
     uint64_t list = 0;
     if (warp == kSelW) {
@@ -163,7 +175,7 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
     }
     __syncthreads();
     if (warp != 0) return;
-    for (int w = 1; w < kSelW; ++w) list_offer(list, lists[w * 32 + lane], lane);
+    for (int w = 1; w < kSelW; ++w) list_merge(list, lists[w * 32 + lane], lane);
 
     if (p.nchunks > 1) {
         uint64_t *mine = p.part_keys + ((int64_t)u * p.nchunks + chunk) * 32;
@@ -182,7 +194,7 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
 #pragma unroll
             for (int j = 0; j < 8; ++j) k[j] = (c0 + j < p.nchunks) ? __ldcg(all + (c0 + j) * 32 + lane) : 0ull;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) list_offer(list, k[j], lane);
+            for (int j = 0; j < 8; ++j) list_merge(list, k[j], lane);
         }
     }
 
@@ -199,10 +211,9 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
     for (int i = lane; i < nw; i += 32) bitmap[i] = 0;
     __syncwarp();
     if (myid >= 0) atomicOr(&bitmap[myid >> 5], 1u << (myid & 31));
-    const int32_t ne = min(p.gamma_n[u], p.k_e);
-    const int32_t *ge = p.gamma_e + (int64_t)u * p.k_e;
-    for (int j = lane; j < ne; j += 32) {
-        const int32_t id = ge[j];
+#pragma unroll
+    for (int i = 0; i < kMaxKe / 32; ++i) {
+        const int32_t id = ge_reg[i];
         if (id >= 0 && id < nb_c) atomicOr(&bitmap[id >> 5], 1u << (id & 31));
     }
     __syncwarp();
