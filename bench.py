@@ -60,6 +60,19 @@ def describe(c, groups):
     return s
 
 
+_PINNED = {}
+
+
+def pinned(nbytes, key):
+    """Pinned host buffer of nbytes, reused across workloads with the same key (pinning is slow)."""
+    t = _PINNED.get(key)
+    if t is None or t.numel() < nbytes:
+        _PINNED.pop(key, None)
+        t = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+        _PINNED[key] = t
+    return t[:nbytes]
+
+
 class Workload:
     """All layers of one configuration: state, prefilled context and per-step inputs on the device.
 
@@ -69,8 +82,8 @@ class Workload:
     sequence still goes through its layers in order.
     """
 
-    def __init__(self, c, n_steps, seed=0, groups=2, layers=None, device="cuda", micro=1, seq_base=0):
-        self.c, self.seed, self.groups, self.seq_base = c, seed, groups, seq_base
+    def __init__(self, c, n_steps, seed=0, groups=2, layers=None, device="cuda", micro=1, seq_base=0, dense=False):
+        self.c, self.seed, self.groups, self.seq_base, self.dense = c, seed, groups, seq_base, dense
         self.L = layers if layers is not None else c["layers"]
         self.B, self.Hq, self.Hkv = c["B"], c["Hq"], c["Hkv"]
         assert self.B % micro == 0, "batch must split evenly into micro-batches"
@@ -86,7 +99,7 @@ class Workload:
             nbytes = nosa.nosa_state_bytes(self.cfg, nosa.BUF_KV_STORE)
             for g in range(min(groups, self.L)):
                 for m in range(micro):
-                    self.host[(g, m)] = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+                    self.host[(g, m)] = pinned(nbytes, (g, m))
         self.layers = [[nosa.NosaLayer(self.cfg, dev, self.host[(l % groups, m)] if self.host else None)
                         for m in range(micro)] for l in range(self.L)]
         self._prefill(dev)
@@ -169,6 +182,9 @@ class Workload:
         lay = self.layers[l][m]
         q, k, v, e = self.views(buf, l, m)
         out = self.out_view(l, m)
+        if self.dense:  # the full-attention comparator: append, then attend to every token
+            return [("append", lambda s: lay.append(k, v, e, 1, None, s)),
+                    ("dense", lambda s: lay.dense_decode(q, out, s))]
         calls = [("append", lambda s: lay.append(k, v, e, 1, None, s)), ("select", lambda s: lay.select(q, s))]
         if self.c["offload"]:
             calls.append(("cache_sync", lambda s: lay.cache_sync(s)))
@@ -202,6 +218,37 @@ class Workload:
         for s in self.streams:
             cur.wait_stream(s)
 
+    def time_steps(self, warmup, steps, first=0):
+        """Device ms per step over `steps` graph-replayed steps (L2 flushed per step if it fits in L2)."""
+        t = first
+        for _ in range(warmup):
+            self.cur.copy_(self.inputs[t])
+            self.launch_step()
+            t += 1
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
+            self.launch_step()
+        torch.cuda.synchronize()
+        small = step_bytes(self) < 2 * L2_BYTES
+        flush = L2Flusher(self.cur.device) if small else None
+        ms = 0.0
+        for _ in range(steps):
+            self.cur.copy_(self.inputs[t])
+            t += 1
+            if flush is not None:
+                flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ms += e0.elapsed_time(e1)
+        del g
+        return ms / steps, t
+
     @property
     def launches_per_step(self):
         # append, select, [cache plan, cache gather], decode
@@ -224,10 +271,14 @@ class L2Flusher:
 
 
 def step_bytes(wl):
-    """Bytes one decode step streams from HBM (pooled keys + selected KV blocks), all layers."""
+    """Bytes one decode step streams from HBM (pooled keys + selected KV blocks, or all KV for
+    the dense comparator), all layers."""
     c = wl.c
     nb = (c["L"] - 1) // 64
-    per_unit = nb * 2048 + (c["k_q"] + c["k_e"] + 1) * (32768 + 256)
+    if getattr(wl, "dense", False):
+        per_unit = (nb + 1) * (32768 + 256)
+    else:
+        per_unit = nb * 2048 + (c["k_q"] + c["k_e"] + 1) * (32768 + 256)
     return wl.L * wl.units * per_unit
 
 
@@ -601,6 +652,36 @@ def run_nosa(args, c, rank, world, dev):
     print(json.dumps(line), flush=True)
 
 
+SWEEP = dict(batch=(1, 8, 32, 128, 256), context=(32768, 131072), k=(32, 64, 128))
+
+
+def run_sweep(args, dev):
+    """One JSON line per sweep point: 1 layer, 16 q / 2 kv heads, batch x context x k (k_e = 0.75 k),
+    KV in device memory and in pinned host memory, against dense decode on identical inputs."""
+    steps, warmup = args.steps, args.warmup
+    for L in SWEEP["context"]:
+        for B in SWEEP["batch"]:
+            base = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=16, k_e=48, steps=warmup + steps)
+            dense = Workload(dict(base, offload=False), warmup + steps + 1, seed=args.seed, dense=True, device=dev)
+            dense_ms, _ = dense.time_steps(warmup, steps)
+            del dense
+            torch.cuda.empty_cache()
+            for k in SWEEP["k"]:
+                for offload in (False, True):
+                    c = dict(base, k_q=k // 4, k_e=3 * k // 4, offload=offload)
+                    wl = Workload(c, warmup + steps + 1, seed=args.seed, device=dev)
+                    ms, _ = wl.time_steps(warmup, steps)
+                    errs = [lay.read_error() for per in wl.layers for lay in per]
+                    del wl
+                    torch.cuda.empty_cache()
+                    print(json.dumps({"sweep": {"batch": B, "context": L, "k": k, "k_q": k // 4, "k_e": 3 * k // 4,
+                                                "kv": "pinned host" if offload else "device"},
+                                      "sparse_tokens_per_s": B / (ms * 1e-3), "sparse_ms_per_step": ms,
+                                      "dense_tokens_per_s": B / (dense_ms * 1e-3), "dense_ms_per_step": dense_ms,
+                                      "speedup_vs_dense": dense_ms / ms, "steps": steps, "warmup": warmup,
+                                      "device_errors": errs}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -617,6 +698,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="batch x context x k sweep against dense decode (one JSON line per point)")
     args = ap.parse_args()
     c = dict(WORKLOADS[args.workload])
     if args.layers is not None:
@@ -634,6 +717,9 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                              device_id=dev)
     nosa.lib()
+    if args.sweep:
+        run_sweep(args, dev)
+        return
     try:
         run_nosa(args, c, rank, world, dev)
     finally:
