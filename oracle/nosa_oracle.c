@@ -54,6 +54,7 @@
 
 typedef struct {
     int32_t D, G, block, sub, k_q, k_e;
+    int32_t ck_bf16;         /* pooled keys stored as bf16 (nearest, ties to even) */
     double scale;
     int64_t cap, L;
     uint16_t *K, *V;         /* [cap][D] bf16 bits */
@@ -117,15 +118,32 @@ void nosa_oracle_unit_free(nosa_oracle_unit *u) {
     free(u->ge_inc); free(u->resident); free(u->prevS); free(u);
 }
 
-/* Compressed key of sub-block s: the fp64 mean of its keys. */
+/*
+ * x rounded to the nearest bf16 value (8 significant bits, fp32 exponent
+ * range), ties to even: the mantissa scaled to [128, 256) is rounded with
+ * rint (the default rounding mode is to nearest, ties to even).
+ */
+double nosa_oracle_round_bf16(double x) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    if (fabs(x) < ldexp(1.0, -126)) return ldexp(rint(ldexp(x, 133)), -133); /* subnormal spacing 2^-133 */
+    int e;
+    double m = frexp(x, &e); /* x = m * 2^e, 0.5 <= |m| < 1 */
+    return ldexp(rint(ldexp(m, 8)), e - 8);
+}
+
+/* Compressed key of sub-block s: the fp64 mean of its keys (rounded to bf16 in that mode). */
 static void compress_sub_block(nosa_oracle_unit *u, int64_t s) {
     for (int32_t d = 0; d < u->D; ++d) {
         double acc = 0.0;
         for (int32_t j = 0; j < u->sub; ++j)
             acc += bf16_to_double(u->K[(s * u->sub + j) * u->D + d]);
-        u->ck[s * u->D + d] = acc / u->sub;
+        double mean = acc / u->sub;
+        u->ck[s * u->D + d] = u->ck_bf16 ? nosa_oracle_round_bf16(mean) : mean;
     }
 }
+
+/* Store pooled keys as bf16 from now on (set before the first append). */
+void nosa_oracle_set_ck_bf16(nosa_oracle_unit *u, int32_t on) { u->ck_bf16 = on != 0; }
 
 /* Block eviction score: max over the block's sub-blocks of the mean eviction logit. */
 static void evict_score_block(nosa_oracle_unit *u, int64_t b) {

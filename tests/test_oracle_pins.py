@@ -8,6 +8,7 @@ known by design, or special cases that reduce to textbook softmax attention.
 import numpy as np
 import pytest
 
+import synth
 from oracle import OracleUnit
 from tests import cases
 
@@ -223,3 +224,51 @@ def test_attend_blocks_matches_own_selection():
     tok = np.concatenate([np.arange(b * 64, b * 64 + 64) for b in (2, 7)])
     want = cases.textbook_attention(q, K, V, e, tok, 1 / np.sqrt(128))
     np.testing.assert_allclose(u.attend_blocks(q, [2, 7]), want, rtol=1e-12, atol=1e-15)
+
+
+def _bf16_neighbours(x):
+    """The two bf16 values around x, found by walking the bf16 bit patterns (brute force)."""
+    import struct
+    f = np.float32(x)
+    bits = int(np.frombuffer(struct.pack("<f", f), np.uint32)[0]) >> 16
+    cands = []
+    for b in range(bits - 2, bits + 3):
+        v = np.frombuffer(struct.pack("<I", (b & 0xFFFF) << 16), np.float32)[0]
+        if np.isfinite(v):
+            cands.append((float(v), b & 0xFFFF))
+    return cands
+
+
+def test_bf16_rounding_is_nearest_ties_to_even():
+    """The oracle's bf16 rounding of pooled keys against a brute-force nearest search."""
+    import oracle
+    rng = np.random.default_rng(0)
+    xs = list(rng.normal(0, 0.05, 4000)) + list(rng.normal(0, 3, 1000))
+    # exact midpoints between neighbouring bf16 values: ties must go to the even pattern
+    xs += [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(0.5 + 2.0 ** -9), 0.0]
+    for x in xs:
+        got = oracle.round_bf16(x)
+        cands = _bf16_neighbours(x)
+        best = min(abs(v - x) for v, _ in cands)
+        near = [(v, b) for v, b in cands if abs(v - x) == best]
+        if len(near) > 1:
+            near = [(v, b) for v, b in near if b % 2 == 0]
+        assert got == near[0][0], (x, got, near)
+
+
+def test_bf16_pooled_keys_are_rounded_means():
+    """With bf16 pooled keys, each stored mean is the rounded fp64 mean (ramp keys: exact closed form)."""
+    import oracle
+    L, D = 16 * 5, 128
+    j = np.arange(L)
+    K = ((j % 16) / 16.0 + 0.01 * (j // 16))[:, None] * np.ones(D)[None, :]
+    Kb = np.asarray(synth.bf16_to_f32(np.asarray([np.float32(v).view(np.uint32) >> 16 for v in K.ravel()],
+                                                   np.uint16)), np.float32).reshape(L, D)
+    Kbits = (Kb.view(np.uint32) >> 16).astype(np.uint16)
+    u = OracleUnit(k_q=1, k_e=1, cap=4096, ck_bf16=True)
+    u.prefill(Kbits, Kbits, np.zeros(L, np.float32))
+    ck = u.ck()
+    means = Kb.astype(np.float64).reshape(5, 16, D).mean(axis=1)
+    want = np.vectorize(oracle.round_bf16)(means)
+    assert np.array_equal(ck, want)
+    assert not np.array_equal(ck, means)  # the rounding really happened
