@@ -57,6 +57,8 @@ def describe(c, groups):
               f"device cache = local + {c['k_q'] + c['k_e']} blocks per (seq, kv head)")
     else:
         s += "KV resident in device memory"
+    if c.get("ck_bf16"):
+        s += ", pooled keys stored bf16"
     return s
 
 
@@ -92,7 +94,8 @@ class Workload:
         self.units_m = self.Bm * self.Hkv
         self.n_steps = n_steps
         self.max_ctx = (c["L"] + n_steps + 63) // 64 * 64
-        self.cfg = nosa.make_config(self.Bm, self.Hq, self.Hkv, c["k_q"], c["k_e"], self.max_ctx, c["offload"])
+        self.cfg = nosa.make_config(self.Bm, self.Hq, self.Hkv, c["k_q"], c["k_e"], self.max_ctx, c["offload"],
+                                    ck_bf16=c.get("ck_bf16", False))
         dev = torch.device(device)
         self.host = {}
         if c["offload"]:
@@ -270,6 +273,11 @@ class L2Flusher:
         self.buf.fill_(1.0)
 
 
+def ck_elem(c):
+    """Bytes per stored pooled-key element: 4 (fp32), or 2 with bf16 pooled keys."""
+    return 2 if c.get("ck_bf16") else 4
+
+
 def step_bytes(wl):
     """Bytes one decode step streams from HBM (pooled keys + selected KV blocks, or all KV for
     the dense comparator), all layers."""
@@ -278,7 +286,7 @@ def step_bytes(wl):
     if getattr(wl, "dense", False):
         per_unit = (nb + 1) * (32768 + 256)
     else:
-        per_unit = nb * 2048 + (c["k_q"] + c["k_e"] + 1) * (32768 + 256)
+        per_unit = nb * 4 * 128 * ck_elem(c) + (c["k_q"] + c["k_e"] + 1) * (32768 + 256)
     return wl.L * wl.units * per_unit
 
 
@@ -427,7 +435,7 @@ def oracle_sample(c, groups, seed, n_units, n_steps, budget_s=25.0):
         V = synth.kv_rows(seed, synth.V_STREAM, kl, b, g, 0, L0 + n_steps)
         E = synth.e_rows(seed, l, b, g, 0, L0 + n_steps)
         Q = np.stack([synth.q_steps(seed, l, b, g * G + h, n_steps)[1] for h in range(G)], axis=1)
-        u = oracle.OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=cap)
+        u = oracle.OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=cap, ck_bf16=c.get("ck_bf16", False))
         u.prefill(K[:L0], V[:L0], E[:L0])
         for t in range(n_steps):
             t0 = time.perf_counter()
@@ -564,7 +572,7 @@ def run_nosa(args, c, rank, world, dev):
     U, Lctx = wl.units_m, c["L"] + step_i
     nb_c = (Lctx - 1) // 64
     algo = {  # algorithmic bytes per launch (one layer of one micro-batch)
-        "select": U * (nb_c * 4 * D * 4 + (c["Hq"] // c["Hkv"]) * D * 2),
+        "select": U * (nb_c * 4 * D * ck_elem(c) + (c["Hq"] // c["Hkv"]) * D * 2),
         "decode": U * nsel_mean * (64 * D * 2 * 2 + 64 * 4) + 2 * wl.Bm * c["Hq"] * D * 2,
         "append": U * (2 * D * 2 + 4),
     }
@@ -639,7 +647,7 @@ def run_nosa(args, c, rank, world, dev):
         "data": "synthetic (seeded counter-based generator: K,V ~ N(0,1)/sqrt(128) bf16, e ~ N(0,1), drifting q)",
         "config": {"workload": f"{args.workload}: " + describe(c, args.host_groups), "layers": c["layers"],
                    "batch": c["B"], "heads_q": c["Hq"], "heads_kv": c["Hkv"], "context": c["L"], "k_q": c["k_q"],
-                   "k_e": c["k_e"], "offload": c["offload"], "host_kv_groups": args.host_groups if c["offload"] else None,
+                   "k_e": c["k_e"], "offload": c["offload"], "pooled_keys": "bf16" if c.get("ck_bf16") else "fp32", "host_kv_groups": args.host_groups if c["offload"] else None,
                    "cuda_graph": graph is not None, "micro_batches": wl.micro,
                    "l2": ("L2 flushed (256 MB write) before every timed step; steps timed one by one" if small else
                           f"inputs larger than L2: each step streams {step_bytes(wl) / 1e9:.2f} GB of pooled keys and KV blocks"),
@@ -661,7 +669,8 @@ def run_sweep(args, dev):
     steps, warmup = args.steps, args.warmup
     for L in SWEEP["context"]:
         for B in SWEEP["batch"]:
-            base = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=16, k_e=48, steps=warmup + steps)
+            base = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=16, k_e=48, steps=warmup + steps,
+                        ck_bf16=args.ck_bf16)
             dense = Workload(dict(base, offload=False), warmup + steps + 1, seed=args.seed, dense=True, device=dev)
             dense_ms, _ = dense.time_steps(warmup, steps)
             del dense
@@ -675,7 +684,8 @@ def run_sweep(args, dev):
                     del wl
                     torch.cuda.empty_cache()
                     print(json.dumps({"sweep": {"batch": B, "context": L, "k": k, "k_q": k // 4, "k_e": 3 * k // 4,
-                                                "kv": "pinned host" if offload else "device"},
+                                                "kv": "pinned host" if offload else "device",
+                                                "pooled_keys": "bf16" if args.ck_bf16 else "fp32"},
                                       "sparse_tokens_per_s": B / (ms * 1e-3), "sparse_ms_per_step": ms,
                                       "dense_tokens_per_s": B / (dense_ms * 1e-3), "dense_ms_per_step": dense_ms,
                                       "speedup_vs_dense": dense_ms / ms, "steps": steps, "warmup": warmup,
@@ -700,8 +710,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="batch x context x k sweep against dense decode (one JSON line per point)")
+    ap.add_argument("--ck-bf16", action="store_true", help="store pooled keys as bf16 instead of fp32")
     args = ap.parse_args()
     c = dict(WORKLOADS[args.workload])
+    if args.ck_bf16:
+        c["ck_bf16"] = True
     if args.layers is not None:
         c["layers"] = args.layers
     world = int(os.environ.get("WORLD_SIZE", "1"))

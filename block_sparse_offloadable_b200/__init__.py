@@ -26,6 +26,7 @@ NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", 
 
 OK, ERR_ARG, ERR_CAPACITY, ERR_PTR, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED, ERR_DEVICE = 0, -1, -2, -3, -4, -5, -6, -7
 EFLAG_CAPACITY, EFLAG_TIMEOUT, EFLAG_NOSLOT, EFLAG_STATE = 1, 2, 4, 8
+FLAG_CK_BF16 = 1
 (BUF_KV_STORE, BUF_EVICT_LOGIT, BUF_CK, BUF_BLK_EVICT, BUF_GAMMA_E, BUF_GAMMA_N, BUF_SEQ_LEN, BUF_CACHE,
  BUF_SLOT_BLOCK, BUF_BLOCK_SLOT, BUF_ERR) = range(11)
 WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC = 0, 1, 2, 3
@@ -57,7 +58,7 @@ class Config(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32), ("sub_block", ctypes.c_int32),
                 ("k_q", ctypes.c_int32), ("k_e", ctypes.c_int32), ("local_blocks", ctypes.c_int32),
                 ("offload", ctypes.c_int32), ("max_ctx", ctypes.c_int64), ("scale", ctypes.c_float),
-                ("reserved", ctypes.c_int32)]
+                ("flags", ctypes.c_int32)]
 
 
 class State(ctypes.Structure):
@@ -117,9 +118,10 @@ def _stream(stream):
 
 
 def make_config(batch, heads_q, heads_kv, k_q, k_e, max_ctx, offload=False, head_dim=128, block=64, sub_block=16,
-                scale=None):
+                scale=None, ck_bf16=False):
     return Config(batch, heads_q, heads_kv, head_dim, block, sub_block, k_q, k_e, 1, int(bool(offload)),
-                  int(max_ctx), float(scale if scale is not None else head_dim ** -0.5), 0)
+                  int(max_ctx), float(scale if scale is not None else head_dim ** -0.5),
+                  FLAG_CK_BF16 if ck_bf16 else 0)
 
 
 # ---- the C entry points, one to one -------------------------------------------------
@@ -218,7 +220,7 @@ class NosaLayer:
         else:
             self.kv_store = dbuf(BUF_KV_STORE)
         self.evict_logit = dbuf(BUF_EVICT_LOGIT, torch.float32)
-        self.ck = dbuf(BUF_CK, torch.float32)
+        self.ck = dbuf(BUF_CK, torch.int16 if cfg.flags & FLAG_CK_BF16 else torch.float32)
         self.blk_evict = dbuf(BUF_BLK_EVICT, torch.float64)
         self.gamma_e = dbuf(BUF_GAMMA_E, torch.int32)
         self.gamma_n = dbuf(BUF_GAMMA_N, torch.int32)

@@ -114,7 +114,7 @@ int kv_tensor_map(CUtensorMap *map, const void *base, int64_t rows) {
 
 int select_nchunks(const nosa_config *c, const Geo &g) {
     if (c->k_q <= 0) return 1;
-    const int cb = select_chunk_blocks((int32_t)g.units, (int32_t)g.nblk);
+    const int cb = select_chunk_blocks((int32_t)g.units, (int32_t)g.nblk, (c->flags & NOSA_FLAG_CK_BF16) != 0);
     int64_t n = (g.nblk - 1 + cb - 1) / cb;
     return n < 1 ? 1 : (int)n;
 }
@@ -200,7 +200,7 @@ int nosa_validate_config(const nosa_config *c) {
     if (!c) return NOSA_ERR_ARG;
     if (c->batch < 1 || c->heads_kv < 1 || c->heads_q < 1 || c->heads_q % c->heads_kv) return NOSA_ERR_ARG;
     if (c->k_q < 0 || c->k_e < 0 || c->k_q + c->k_e < 1 || c->max_ctx <= 0 ||
-        c->max_ctx % 64 || c->reserved != 0 || !(c->scale > 0.f) || !isfinite(c->scale))
+        c->max_ctx % 64 || (c->flags & ~NOSA_FLAG_CK_BF16) != 0 || !(c->scale > 0.f) || !isfinite(c->scale))
         return NOSA_ERR_ARG;
     if (c->offload != 0 && c->offload != 1) return NOSA_ERR_ARG;
     if (c->head_dim != kD || c->block != kBlock || c->sub_block != kSub || c->local_blocks != 1)
@@ -222,7 +222,7 @@ size_t nosa_state_bytes(const nosa_config *c, int which) {
     switch (which) {
     case NOSA_BUF_KV_STORE: return u * g.nblk * kBlockBytes;
     case NOSA_BUF_EVICT_LOGIT: return u * c->max_ctx * sizeof(float);
-    case NOSA_BUF_CK: return u * g.nsub * kD * sizeof(float);
+    case NOSA_BUF_CK: return u * g.nsub * kD * ((c->flags & NOSA_FLAG_CK_BF16) ? 2 : sizeof(float));
     case NOSA_BUF_BLK_EVICT: return u * g.nblk * sizeof(double);
     case NOSA_BUF_GAMMA_E: return u * (c->k_e > 0 ? c->k_e : 1) * sizeof(int32_t);
     case NOSA_BUF_GAMMA_N:
@@ -284,7 +284,7 @@ int nosa_compress_append(const nosa_config *c, const nosa_state *st, const uint1
     p.max_ctx = c->max_ctx;
     p.nblk = (int32_t)g.nblk; p.nsub = (int32_t)g.nsub; p.nslots = (int32_t)g.nslots;
     p.units = (int32_t)g.units; p.heads_kv = c->heads_kv; p.k_e = c->k_e;
-    p.offload = c->offload; p.T = T;
+    p.offload = c->offload; p.T = T; p.ck_bf16 = (c->flags & NOSA_FLAG_CK_BF16) != 0;
     return launch_append(p, static_cast<cudaStream_t>(stream));
 }
 
@@ -305,8 +305,9 @@ int nosa_select(const nosa_config *c, const nosa_state *st, const uint16_t *q, i
     p.sel = sel; p.nsel = nsel; p.gq = c->k_q > 0 ? gq : nullptr; p.err = st->err;
     p.nsub = (int32_t)g.nsub; p.nblk = (int32_t)g.nblk; p.G = (int32_t)g.G; p.units = (int32_t)g.units;
     p.nchunks = select_nchunks(c, g);
-    p.chunk_blocks = c->k_q > 0 ? select_chunk_blocks(p.units, p.nblk) : p.nblk;
+    p.chunk_blocks = c->k_q > 0 ? select_chunk_blocks(p.units, p.nblk, (c->flags & NOSA_FLAG_CK_BF16) != 0) : p.nblk;
     p.k_q = c->k_q; p.k_e = c->k_e; p.max_sel = (int32_t)g.max_sel; p.scale = c->scale;
+    p.ck_bf16 = (c->flags & NOSA_FLAG_CK_BF16) != 0;
     if (p.nchunks > 1) {
         p.counter = static_cast<int32_t *>(ws);
         p.part_keys = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(ws) +

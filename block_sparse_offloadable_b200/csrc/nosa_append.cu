@@ -15,6 +15,22 @@
 
 namespace nosa {
 
+// Store this lane's 4 pooled-key dims (fp64 means) as fp32, or as bf16 rounded once from fp64.
+__device__ __forceinline__ void store_ck(const AppendParams &p, int64_t row, int lane, double a0, double a1,
+                                         double a2, double a3) {
+    if (p.ck_bf16) {
+        __nv_bfloat16 b0 = __double2bfloat16(a0), b1 = __double2bfloat16(a1);
+        __nv_bfloat16 b2 = __double2bfloat16(a2), b3 = __double2bfloat16(a3);
+        uint2 w;
+        w.x = (uint32_t)*reinterpret_cast<uint16_t *>(&b0) | ((uint32_t)*reinterpret_cast<uint16_t *>(&b1) << 16);
+        w.y = (uint32_t)*reinterpret_cast<uint16_t *>(&b2) | ((uint32_t)*reinterpret_cast<uint16_t *>(&b3) << 16);
+        reinterpret_cast<uint2 *>(static_cast<uint16_t *>(p.ck) + row * kD)[lane] = w;
+    } else {
+        reinterpret_cast<float4 *>(static_cast<float *>(p.ck) + row * kD)[lane] =
+            make_float4((float)a0, (float)a1, (float)a2, (float)a3);
+    }
+}
+
 // Warp-cooperative argmin over Gamma_e by (E ascending, block id descending):
 // the member that leaves when a better block arrives.
 __device__ __forceinline__ void gamma_e_worst(const int32_t *ge, int32_t ne, const double *E,
@@ -103,9 +119,7 @@ __global__ void __launch_bounds__(128) append_decode_kernel(const AppendParams p
         const uint2 v = reinterpret_cast<const uint2 *>(p.k_new + (int64_t)u * kD)[lane];
         acc0 += bf16_lo(v.x); acc1 += bf16_hi(v.x);
         acc2 += bf16_lo(v.y); acc3 += bf16_hi(v.y);
-        float4 out = make_float4((float)(acc0 / kSub), (float)(acc1 / kSub), (float)(acc2 / kSub),
-                                 (float)(acc3 / kSub));
-        reinterpret_cast<float4 *>(p.ck + ((int64_t)u * p.nsub + s) * kD)[lane] = out;
+        store_ck(p, (int64_t)u * p.nsub + s, lane, acc0 / kSub, acc1 / kSub, acc2 / kSub, acc3 / kSub);
     }
 
     // block complete: E_b = max over its sub-blocks of the mean eviction logit (fp64)
@@ -210,9 +224,7 @@ __global__ void __launch_bounds__(256) prefill_pool_kernel(const AppendParams p)
                 a0 += bf16_lo(v.x); a1 += bf16_hi(v.x);
                 a2 += bf16_lo(v.y); a3 += bf16_hi(v.y);
             }
-            float4 out = make_float4((float)(a0 / kSub), (float)(a1 / kSub), (float)(a2 / kSub),
-                                     (float)(a3 / kSub));
-            reinterpret_cast<float4 *>(p.ck + ((int64_t)u * p.nsub + (t0 >> 4)) * kD)[lane] = out;
+            store_ck(p, (int64_t)u * p.nsub + (t0 >> 4), lane, a0 / kSub, a1 / kSub, a2 / kSub, a3 / kSub);
         }
         if ((blk + 1) * kBlock <= len) {
             double m = -__longlong_as_double(0x7FF0000000000000ll);

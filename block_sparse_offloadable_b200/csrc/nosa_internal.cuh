@@ -14,7 +14,7 @@ struct AppendParams {
     uint8_t *store;          // device address of the KV store (device memory or mapped host)
     uint8_t *cache;          // offload cache or null
     float *e_store;          // [u][max_ctx]
-    float *ck;               // [u][nsub][D]
+    void *ck;                // [u][nsub][D] fp32, or bf16 when ck_bf16
     double *blk_evict;       // [u][nblk]
     int32_t *gamma_e;        // [u][k_e]
     int32_t *gamma_n;        // [u]
@@ -23,12 +23,12 @@ struct AppendParams {
     int32_t *block_slot;     // [u][nblk]
     uint32_t *err;
     int64_t max_ctx;
-    int32_t nblk, nsub, nslots, units, heads_kv, k_e, offload, T;
+    int32_t nblk, nsub, nslots, units, heads_kv, k_e, offload, T, ck_bf16;
 };
 
 struct SelectParams {
     const uint16_t *q;        // [B][Hq][D]
-    const float *ck;          // [u][nsub][D]
+    const void *ck;           // [u][nsub][D] fp32, or bf16 when ck_bf16
     const int32_t *gamma_e;   // [u][k_e]
     const int32_t *gamma_n;   // [u]
     const int32_t *seq_len;   // [u]
@@ -38,7 +38,7 @@ struct SelectParams {
     uint64_t *part_keys;      // [u][nchunks][32]
     int32_t *counter;         // [u]
     uint32_t *err;
-    int32_t nsub, nblk, G, units, nchunks, chunk_blocks, k_q, k_e, max_sel;
+    int32_t nsub, nblk, G, units, nchunks, chunk_blocks, k_q, k_e, max_sel, ck_bf16;
     float scale;
 };
 
@@ -82,7 +82,7 @@ int launch_cache_sync(const CacheParams &p, cudaStream_t stream);
 int launch_decode(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t stream);
 
 // Launch geometry, shared by the launchers and the workspace-size queries.
-int select_chunk_blocks(int32_t units, int32_t nblk);
+int select_chunk_blocks(int32_t units, int32_t nblk, bool ck_bf16);
 int decode_ctas();
 constexpr int kMaxUnits = 2048;  // (seq, kv head) units per call: the decode kernel's prefix sums live in shared memory
 

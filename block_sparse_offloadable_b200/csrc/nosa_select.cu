@@ -7,34 +7,53 @@
 // budget k_q and a query-agnostic budget k_e); gist.science summary,
 // "Mecanisme de double selection".
 //
-// Design.  The only large operand is the fp32 compressed-key array of a unit
-// (32 B per token: 4 MiB per unit at 128K context), read once per step: the
-// kernel is a streaming GEMV against q_hat = sum of the group's query heads,
-// bound by HBM bandwidth.  Each CTA owns a contiguous chunk of candidate
-// blocks.  One producer thread streams the chunk into a ring of shared-memory
-// stages with bulk asynchronous copies (cp.async.bulk, completion on
-// mbarriers); consumer warps read 32 sub-block rows per stage with 16-byte
-// shared loads, reduce the 32 partial dot products with a 31-shuffle
-// transpose-reduction (each lane ends with one sub-block), max-pool groups of
-// four lanes to block scores, and keep a warp-wide sorted top-32 list of
-// (score, block) keys.  The per-chunk lists go to the workspace; the last CTA
-// of the unit to finish (atomic counter, no waiting) merges them into Gamma_q,
-// forms the union with Gamma_e through a block bitmap, appends the local block
-// and writes the ascending selection.
+// Design.  The only large operand is the compressed-key array of a unit (fp32:
+// 32 B per token, 4 MiB per unit at 128K context; bf16: half that), read once
+// per step: the kernel is a streaming GEMV against q_hat = sum of the group's
+// query heads, bound by HBM bandwidth.  Each CTA owns a contiguous chunk of
+// candidate blocks.  One producer thread streams the chunk into a ring of
+// shared-memory stages with bulk asynchronous copies (cp.async.bulk,
+// completion on mbarriers); consumer warps read 32 sub-block rows per stage
+// (each lane 4 dims of a row: a 16-byte fp32 or 8-byte bf16 shared load),
+// reduce the 32 partial dot products with a 31-shuffle transpose-reduction
+// (each lane ends with one sub-block), max-pool groups of four lanes to block
+// scores, and keep a warp-wide sorted top-32 list of (score, block) keys.  The
+// per-chunk lists go to the workspace; the last CTA of the unit to finish
+// (atomic counter, no waiting) merges them into Gamma_q, forms the union with
+// Gamma_e through a block bitmap, appends the local block and writes the
+// ascending selection.
 #include "nosa_internal.cuh"
 
 namespace nosa {
 
 namespace {
 constexpr int kSelW = 4;    // consumer warps
-constexpr int kSelS = 4;    // stages
-constexpr int kSelSB = 8;   // blocks per stage (32 sub-block rows, 16 KiB)
-constexpr int kStageBytes = kSelSB * kSubPerBlock * kD * 4;
+constexpr int kSelSB = 8;   // blocks per stage (32 sub-block rows)
 constexpr int kCtasPerSm = 3;
+constexpr int kMaxChunks = 64;  // select_chunk_blocks keeps chunks per unit below this
+
+// Stage geometry per stored key type: 64 KiB in flight per CTA either way
+// (fp32: 4 stages of 16 KiB; bf16: 8 stages of 8 KiB).
+template <typename T> struct SelGeo;
+template <> struct SelGeo<float> { static constexpr int kElem = 4, kStages = 4; };
+template <> struct SelGeo<__nv_bfloat16> { static constexpr int kElem = 2, kStages = 8; };
+template <typename T> __host__ __device__ constexpr int stage_bytes() { return kSelSB * kSubPerBlock * kD * SelGeo<T>::kElem; }
 // Stage s is always consumed by warp s % kSelW, so every mbarrier waiter waits
 // its phases in order (parity waits cannot tell phase p from p + 2).
-static_assert(kSelS % kSelW == 0, "each stage must have a single consumer warp");
-constexpr int kMaxChunks = 64;  // select_chunk_blocks keeps chunks per unit below this
+static_assert(SelGeo<float>::kStages % kSelW == 0, "each stage must have a single consumer warp");
+static_assert(SelGeo<__nv_bfloat16>::kStages % kSelW == 0, "each stage must have a single consumer warp");
+
+// This lane's 4 dims of one pooled-key row in shared memory.
+__device__ __forceinline__ float4 row4(const uint8_t *tile, int row, int lane, float *) {
+    return lds128f(tile + row * (kD * 4) + lane * 16);
+}
+__device__ __forceinline__ float4 row4(const uint8_t *tile, int row, int lane, __nv_bfloat16 *) {
+    uint2 w;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(w.x), "=r"(w.y)
+                 : "r"(smem_u32(tile + row * (kD * 2) + lane * 8)));
+    return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+}
 
 // One level of the transpose-reduction: lanes exchange the half they do not keep.
 template <int N>
@@ -48,25 +67,31 @@ __device__ __forceinline__ void reduce_level(float (&v)[32], int lane, int o) {
     }
 }
 
+template <typename T>
 size_t select_smem_bytes(int32_t nblk) {
-    return (size_t)kSelS * kStageBytes + 2 * kSelS * sizeof(uint64_t) +
-           kSelW * 32 * sizeof(uint64_t) + ((size_t)nblk / 32 + 1) * sizeof(uint32_t);
+    constexpr int S = SelGeo<T>::kStages;
+    return (size_t)S * stage_bytes<T>() + 2 * S * sizeof(uint64_t) + kSelW * 32 * sizeof(uint64_t) +
+           ((size_t)nblk / 32 + 1) * sizeof(uint32_t);
 }
 }  // namespace
 
-int select_chunk_blocks(int32_t units, int32_t nblk) {
-    // candidates per unit are at most nblk - 1; per-CTA fixed cost ~ 32 blocks
-    // (pipeline fill, the list merges, the atomic hand-off)
+int select_chunk_blocks(int32_t units, int32_t nblk, bool ck_bf16) {
+    // candidates per unit are at most nblk - 1; per-CTA fixed cost (pipeline
+    // fill, the list merges, the atomic hand-off) ~ the time of 32 fp32 blocks,
+    // i.e. of 64 bf16 blocks
     const int64_t work = nblk > 1 ? nblk - 1 : 1;
     int64_t nmax = (work + kSelSB - 1) / kSelSB;
     if (nmax > kMaxChunks) nmax = kMaxChunks;
-    const int n = best_chunks(units, work, (int64_t)kNumSms * kCtasPerSm, 32, nmax);
+    const int n = best_chunks(units, work, (int64_t)kNumSms * kCtasPerSm, ck_bf16 ? 64 : 32, nmax);
     int64_t per = (work + n - 1) / n;
     per = (per + kSelSB - 1) / kSelSB * kSelSB;
     return (int)per;
 }
 
+template <typename T>
 __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectParams p) {
+    constexpr int kSelS = SelGeo<T>::kStages;
+    constexpr int kStageBytes = stage_bytes<T>();
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *tiles = smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(tiles + kSelS * kStageBytes);
@@ -114,11 +139,11 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
                     break;
                 }
                 const int32_t bs = b0 + i * kSelSB;
-                const uint32_t bytes = (uint32_t)min(kSelSB, b1 - bs) * (kSubPerBlock * kD * 4);
+                const uint32_t bytes = (uint32_t)min(kSelSB, b1 - bs) * (kSubPerBlock * kD * SelGeo<T>::kElem);
                 mbar_arrive_expect_tx(&full[s], bytes);
                 bulk_load(tiles + s * kStageBytes,
-                          p.ck + ((int64_t)u * p.nsub + (int64_t)bs * kSubPerBlock) * kD, bytes,
-                          &full[s]);
+                          static_cast<const T *>(p.ck) + ((int64_t)u * p.nsub + (int64_t)bs * kSubPerBlock) * kD,
+                          bytes, &full[s]);
             }
             // never leave with copies in flight
             for (int i = max(0, nstage - kSelS); i < nstage; ++i)
@@ -147,11 +172,11 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
                 set_error(p.err, NOSA_EFLAG_TIMEOUT);
                 break;
             }
-            const uint8_t *t = tiles + s * kStageBytes + lane * 16;
+            const uint8_t *t = tiles + s * kStageBytes;
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float4 k = lds128f(t + j * (kD * 4));
+                const float4 k = row4(t, j, lane, static_cast<T *>(nullptr));
                 v[j] = fmaf(qv.w, k.w, fmaf(qv.z, k.z, fmaf(qv.y, k.y, qv.x * k.x)));
             }
             __syncwarp();
@@ -243,14 +268,19 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
     for (int i = total + 1 + lane; i < p.max_sel; i += 32) sel[i] = -1;
 }
 
-int launch_select(const SelectParams &p, cudaStream_t stream) {
-    const size_t smem = select_smem_bytes(p.nblk);
-    if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <typename T>
+int launch_select_t(const SelectParams &p, cudaStream_t stream) {
+    const size_t smem = select_smem_bytes<T>(p.nblk);
+    if (cudaFuncSetAttribute(select_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return NOSA_ERR_CUDA;
     dim3 grid(p.nchunks, p.units);
-    select_kernel<<<grid, (kSelW + 1) * 32, smem, stream>>>(p);
+    select_kernel<T><<<grid, (kSelW + 1) * 32, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? NOSA_OK : NOSA_ERR_CUDA;
+}
+
+int launch_select(const SelectParams &p, cudaStream_t stream) {
+    return p.ck_bf16 ? launch_select_t<__nv_bfloat16>(p, stream) : launch_select_t<float>(p, stream);
 }
 
 }  // namespace nosa

@@ -77,8 +77,14 @@ typedef struct nosa_config {
     int32_t offload;      /* 0: KV store in device memory; 1: KV store in host memory + device block cache */
     int64_t max_ctx;      /* capacity in tokens per sequence */
     float scale;          /* softmax scale of q.k (normally 1/sqrt(D)) */
-    int32_t reserved;     /* must be 0 */
+    int32_t flags;        /* NOSA_FLAG_* bits; 0 = defaults */
 } nosa_config;
+
+/*
+ * Pooled keys stored as bf16 (the fp64 sub-block mean rounded to the nearest
+ * bf16, ties to even) instead of fp32: half the bytes nosa_select streams.
+ */
+#define NOSA_FLAG_CK_BF16 0x1
 
 /*
  * Per-layer state.  Every buffer is caller-owned; nosa_state_bytes(cfg, NOSA_BUF_x)
@@ -87,7 +93,8 @@ typedef struct nosa_config {
  *   kv_store    bf16 [u][nblk][2][64][D]; [..][0] = keys, [..][1] = values.
  *               Device memory if offload == 0, host memory if offload == 1.
  *   evict_logit fp32 [u][max_ctx]   per-token eviction logit e_j (device)
- *   ck          fp32 [u][nsub][D]   compressed keys: mean of each 16-token sub-block (device)
+ *   ck          fp32 [u][nsub][D]   compressed keys: mean of each 16-token sub-block (device);
+ *               bf16 [u][nsub][D] with NOSA_FLAG_CK_BF16
  *   blk_evict   fp64 [u][nblk]      block eviction score E_b, pre-exponential (device)
  *   gamma_e     int32 [u][k_e]      Gamma_e block ids, ascending (device)
  *   gamma_n     int32 [u]           |Gamma_e| (device)
@@ -101,7 +108,7 @@ typedef struct nosa_config {
 typedef struct nosa_state {
     void *kv_store;
     float *evict_logit;
-    float *ck;
+    void *ck;
     double *blk_evict;
     int32_t *gamma_e;
     int32_t *gamma_n;
@@ -168,7 +175,7 @@ int nosa_state_init(const nosa_config *cfg, const nosa_state *st, void *stream);
  * For each unit: stores the rows at position L (offload: into the device cache
  * slot of the local block, and written through to the host store); when a
  * 16-token sub-block completes, stores its mean key (fp64 sum of the bf16
- * keys, stored fp32); when a 64-token block completes, stores E_b = max over
+ * keys, stored fp32, or rounded to bf16 with NOSA_FLAG_CK_BF16); when a 64-token block completes, stores E_b = max over
  * its sub-blocks of the mean eviction logit (fp64); when a block becomes a
  * candidate, it enters Gamma_e if |Gamma_e| < k_e, or replaces the member with
  * the lowest E if its E is strictly higher (the member is then dropped for

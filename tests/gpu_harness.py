@@ -23,7 +23,7 @@ MAX_ABS, MEAN_ABS, REL_L2 = 1e-2, 1e-3, 1e-2
 
 class Scenario:
     def __init__(self, B, Hq, Hkv, k_q, k_e, L0, steps, offload=False, seed=0, layer=0, lens=None,
-                 max_ctx=None, dense=False):
+                 max_ctx=None, dense=False, ck_bf16=False):
         self.B, self.Hq, self.Hkv, self.k_q, self.k_e = B, Hq, Hkv, k_q, k_e
         self.G = Hq // Hkv
         self.units = B * Hkv
@@ -32,9 +32,11 @@ class Scenario:
         self.Lmax = max(self.lens) + steps
         self.max_ctx = max_ctx or ((self.Lmax + 63) // 64 * 64 + 64)
         self.dense = dense
+        self.ck_bf16 = ck_bf16
 
     def cfg(self):
-        return nosa.make_config(self.B, self.Hq, self.Hkv, self.k_q, self.k_e, self.max_ctx, self.offload)
+        return nosa.make_config(self.B, self.Hq, self.Hkv, self.k_q, self.k_e, self.max_ctx, self.offload,
+                                ck_bf16=self.ck_bf16)
 
 
 def unit_data(sc):
@@ -102,6 +104,7 @@ def run_gpu(sc, data):
     torch.cuda.synchronize()
     res["err"] = lay.read_error()
     res["seq_len"] = lay.seq_len.cpu().numpy()
+    res["ck"] = lay.ck.cpu().numpy()
     return res
 
 
@@ -165,7 +168,7 @@ def compare(sc, data, gpu, units=None, report=None):
     for u in units:
         b, g = divmod(u, sc.Hkv)
         n0 = sc.lens[b]
-        o = OracleUnit(G=sc.G, k_q=sc.k_q, k_e=sc.k_e, cap=sc.max_ctx)
+        o = OracleUnit(G=sc.G, k_q=sc.k_q, k_e=sc.k_e, cap=sc.max_ctx, ck_bf16=sc.ck_bf16)
         if n0 > 0:
             o.prefill(K[u, :n0], V[u, :n0], E[u, :n0])
         history_ok = True

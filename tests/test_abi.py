@@ -42,6 +42,10 @@ def test_validate_config(L):
     assert nosa.nosa_validate_config(cfg(head_dim=64)) == nosa.ERR_UNSUPPORTED
     assert nosa.nosa_validate_config(cfg(max_ctx=1 << 21)) == nosa.ERR_CAPACITY
     assert nosa.nosa_validate_config(cfg(batch=1024, max_ctx=1 << 20)) == nosa.ERR_CAPACITY
+    assert nosa.nosa_validate_config(cfg(ck_bf16=True)) == nosa.OK
+    bad = cfg()
+    bad.flags = 2  # an undefined flag bit
+    assert nosa.nosa_validate_config(bad) == nosa.ERR_ARG
 
 
 def test_state_sizes(L):
@@ -56,6 +60,7 @@ def test_state_sizes(L):
     assert nosa.nosa_state_bytes(co, nosa.BUF_CACHE) == u * (16 + 48 + 2) * 32768
     assert nosa.nosa_state_bytes(co, nosa.BUF_BLOCK_SLOT) == u * nblk * 4
     assert nosa.nosa_state_bytes(cfg(max_ctx=100), nosa.BUF_CK) == 0  # invalid config
+    assert nosa.nosa_state_bytes(cfg(ck_bf16=True), nosa.BUF_CK) == u * (8192 // 16) * 128 * 2
 
 
 def test_workspace_sizes_cover_chunks(L):

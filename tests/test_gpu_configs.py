@@ -72,7 +72,7 @@ def run_config(c, steps, seqs=None, seed=0, micro=1, dense_step=None, name=None)
         V = synth.kv_rows(seed, synth.V_STREAM, wl.kv_layer(0), b, g, 0, L0 + steps)
         E = synth.e_rows(seed, 0, b, g, 0, L0 + steps)
         Q = np.stack([synth.q_steps(seed, 0, b, g * G + h, steps)[1] for h in range(G)], axis=1)
-        o = OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=wl.max_ctx)
+        o = OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=wl.max_ctx, ck_bf16=c.get("ck_bf16", False))
         o.prefill(K[:L0], V[:L0], E[:L0])
         ok = True
         for t in range(steps):
