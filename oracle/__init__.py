@@ -53,6 +53,7 @@ def lib():
         L.nosa_oracle_violations.argtypes = [P, P]
         L.nosa_oracle_attend_blocks.argtypes = [P, P, P, ctypes.c_int32, P]
         L.nosa_oracle_set_ck_bf16.argtypes = [P, ctypes.c_int32]
+        L.nosa_oracle_set_fill.argtypes = [P, ctypes.c_int32]
         L.nosa_oracle_round_bf16.argtypes = [ctypes.c_double]
         L.nosa_oracle_round_bf16.restype = ctypes.c_double
         _lib = L
@@ -71,7 +72,8 @@ def round_bf16(x):
 class OracleUnit:
     """One (sequence, kv head) unit: its KV history, pooled keys and selection state."""
 
-    def __init__(self, D=128, G=1, block=64, sub=16, k_q=16, k_e=48, scale=None, cap=8192, ck_bf16=False):
+    def __init__(self, D=128, G=1, block=64, sub=16, k_q=16, k_e=48, scale=None, cap=8192, ck_bf16=False,
+                 fill=False):
         self.D, self.G, self.block, self.sub, self.k_q, self.k_e = D, G, block, sub, k_q, k_e
         self.scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
         self.cap = cap
@@ -80,6 +82,8 @@ class OracleUnit:
             raise ValueError("oracle: bad unit parameters")
         if ck_bf16:
             lib().nosa_oracle_set_ck_bf16(self._u, 1)
+        if fill:
+            lib().nosa_oracle_set_fill(self._u, 1)
 
     def __del__(self):
         if getattr(self, "_u", None) and _lib is not None:

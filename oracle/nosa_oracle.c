@@ -28,6 +28,11 @@
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - Gamma_q and Gamma_e are independent top-k's whose union is taken.
+ *     Alternative reading, "fill" (item 4 of the same summary: query-aware
+ *     blocks first, the remainder filled by query-agnostic ones): Gamma_e is
+ *     the top-k_e by E among the candidates that are neither in Gamma_q nor
+ *     dropped, where a block is dropped for good at the first step at which
+ *     no component selects it.  Sel then has up to k blocks, disjoint parts.
  *   - A query-group (GQA) score is the sum over its q heads of q_h . kbar.
  *   - Sub-blocks are 16 aligned, non-overlapping tokens; 4 per block.  The
  *     eviction score of a block is the same two-stage pooling applied to the
@@ -55,6 +60,7 @@
 typedef struct {
     int32_t D, G, block, sub, k_q, k_e;
     int32_t ck_bf16;         /* pooled keys stored as bf16 (nearest, ties to even) */
+    int32_t fill;            /* "fill" reading of the Gamma_q / Gamma_e combination */
     double scale;
     int64_t cap, L;
     uint16_t *K, *V;         /* [cap][D] bf16 bits */
@@ -144,6 +150,8 @@ static void compress_sub_block(nosa_oracle_unit *u, int64_t s) {
 
 /* Store pooled keys as bf16 from now on (set before the first append). */
 void nosa_oracle_set_ck_bf16(nosa_oracle_unit *u, int32_t on) { u->ck_bf16 = on != 0; }
+
+void nosa_oracle_set_fill(nosa_oracle_unit *u, int32_t on) { u->fill = on != 0; }
 
 /* Block eviction score: max over the block's sub-blocks of the mean eviction logit. */
 static void evict_score_block(nosa_oracle_unit *u, int64_t b) {
@@ -312,7 +320,7 @@ int nosa_oracle_step(nosa_oracle_unit *u, const uint16_t *k, const uint16_t *v, 
     int32_t nb_c = n_candidates(u);
     int32_t local = (int32_t)((u->L - 1) / u->block);
     int new_local = ((u->L - 1) % u->block) == 0;
-    if (new_local && local >= 1) gamma_e_insert(u, local - 1);
+    if (new_local && local >= 1 && !u->fill) gamma_e_insert(u, local - 1);
 
     double *s = (double *)malloc(sizeof(double) * (size_t)(nb_c + 1));
     block_scores(u, q, nb_c, s);
@@ -320,12 +328,28 @@ int nosa_oracle_step(nosa_oracle_unit *u, const uint16_t *k, const uint16_t *v, 
 
     int32_t n_q = top_k(s, nb_c, u->k_q, gq);
     int32_t *ge_rank = (int32_t *)malloc(sizeof(int32_t) * (size_t)(u->k_e + 1));
-    int32_t n_e = top_k(u->E, nb_c, u->k_e, ge_rank);
+    int32_t n_e;
+    if (!u->fill) {
+        n_e = top_k(u->E, nb_c, u->k_e, ge_rank);
+    } else {
+        /* fill: top-k_e by E over the candidates outside Gamma_q not yet dropped */
+        double *Ef = (double *)malloc(sizeof(double) * (size_t)(nb_c + 1));
+        unsigned char *in_q = (unsigned char *)calloc((size_t)(nb_c + 1), 1);
+        for (int32_t i = 0; i < n_q; ++i) in_q[gq[i]] = 1;
+        int32_t n_elig = 0;
+        for (int32_t b = 0; b < nb_c; ++b) {
+            int elig = !in_q[b] && !u->dropped[b];
+            Ef[b] = elig ? u->E[b] : -INFINITY;
+            n_elig += elig;
+        }
+        n_e = top_k(Ef, nb_c, u->k_e < n_elig ? u->k_e : n_elig, ge_rank);
+        free(Ef); free(in_q);
+    }
     memcpy(ge, ge_rank, sizeof(int32_t) * (size_t)n_e);
     qsort(ge, (size_t)n_e, sizeof(int32_t), cmp_int);
 
-    /* invariant (iii): incremental Gamma_e equals the brute-force one */
-    {
+    /* invariant (iii), union reading: incremental Gamma_e equals the brute-force one */
+    if (!u->fill) {
         int32_t cnt = 0, mismatch = 0;
         for (int32_t b = 0; b < nb_c; ++b) cnt += u->ge_inc[b];
         if (cnt != n_e) mismatch = 1;
@@ -333,16 +357,19 @@ int nosa_oracle_step(nosa_oracle_unit *u, const uint16_t *k, const uint16_t *v, 
             if (!u->ge_inc[ge[i]]) mismatch = 1;
         if (mismatch) u->viol_incremental++;
     }
-    /* invariant (ii): no dropped block re-enters Gamma_e; then mark the new drops */
+    /* invariant (ii): no dropped block re-enters Gamma_e; then mark the new drops
+       (union: every candidate outside Gamma_e; fill: every candidate outside Sel) */
     {
-        unsigned char *in_e = (unsigned char *)calloc((size_t)(nb_c + 1), 1);
+        unsigned char *keep = (unsigned char *)calloc((size_t)(nb_c + 1), 1);
         for (int32_t i = 0; i < n_e; ++i) {
             if (u->dropped[ge[i]]) u->viol_reselect++;
-            in_e[ge[i]] = 1;
+            keep[ge[i]] = 1;
         }
+        if (u->fill)
+            for (int32_t i = 0; i < n_q; ++i) keep[gq[i]] = 1;
         for (int32_t b = 0; b < nb_c; ++b)
-            if (!in_e[b]) u->dropped[b] = 1;
-        free(in_e);
+            if (!keep[b]) u->dropped[b] = 1;
+        free(keep);
     }
 
     /* Sel = Gamma_q ∪ Gamma_e, ascending; S = Sel ∪ {local} */

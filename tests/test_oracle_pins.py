@@ -272,3 +272,99 @@ def test_bf16_pooled_keys_are_rounded_means():
     want = np.vectorize(oracle.round_bf16)(means)
     assert np.array_equal(ck, want)
     assert not np.array_equal(ck, means)  # the rounding really happened
+
+
+def _fixture_query(spec, qspec):
+    s = dict(spec, q=qspec)
+    return cases.build_fixture(s)[3]
+
+
+@pytest.mark.parametrize("fill", [True, False])
+def test_fill_golden_sequence(fill):
+    """Fill reading, hand-derived over four steps: the remainder is filled from the not-yet-dropped
+    blocks outside Gamma_q, a dropped block stays dropped, and Sel may hold fewer than k blocks.
+    The union reading on the same input differs at the first step."""
+    spec = cases.load_fixture("fill_sticky_drop.json")
+    K, V, e, _ = cases.build_fixture(spec)
+    u = OracleUnit(D=spec["D"], G=spec["G"], block=spec["block"], sub=spec["sub"], k_q=spec["k_q"],
+                   k_e=spec["k_e"], cap=64 * 64, fill=fill)
+    u.prefill(K, V, e)
+    z = np.zeros(spec["D"], np.uint16)
+    steps = spec["steps"] if fill else spec["steps"][:1]
+    for i, st in enumerate(steps):
+        r = u.step(z, z, 0.0, _fixture_query(spec, st["q"]))
+        want = st if fill else spec["union_step1"]
+        assert r["gq"].tolist() == st["expect_gq"], i
+        assert r["ge"].tolist() == want["expect_ge"], i
+        assert r["sel"].tolist() == want["expect_sel"], i
+    v = u.violations()
+    assert v["gamma"] == 0 and v["reselect"] == 0
+
+
+def test_fill_with_no_query_budget_equals_union():
+    """With k_q = 0 nothing is excluded by Gamma_q, so the fill and union readings coincide step by step."""
+    L0, steps = 64 * 30 + 9, 140
+    K, V, e = cases.synthetic_unit(5, 0, 0, 0, L0 + steps)
+    Q = cases.synthetic_queries(5, 0, 0, 0, 2, steps)
+    a = OracleUnit(G=2, k_q=0, k_e=7, cap=4096)
+    b = OracleUnit(G=2, k_q=0, k_e=7, cap=4096, fill=True)
+    a.prefill(K[:L0], V[:L0], e[:L0])
+    b.prefill(K[:L0], V[:L0], e[:L0])
+    for t in range(steps):
+        ra = a.step(K[L0 + t], V[L0 + t], float(e[L0 + t]), Q[t])
+        rb = b.step(K[L0 + t], V[L0 + t], float(e[L0 + t]), Q[t])
+        assert np.array_equal(ra["sel"], rb["sel"]) and np.array_equal(ra["ge"], rb["ge"]), t
+        assert np.array_equal(ra["o"], rb["o"])
+
+
+@pytest.mark.parametrize("G,k_q,k_e", [(2, 4, 6), (1, 8, 3)])
+def test_fill_rules_checked_from_history(G, k_q, k_e):
+    """Fill reading, checked step by step against the selection history alone: Gamma_e is disjoint
+    from Gamma_q, holds no block that some earlier step left unselected, is the best of the eligible
+    blocks by E (ties to the lower id) and is as large as k_e allows; gamma(t) >= k_e/k holds."""
+    L0, steps = 64 * 24 + 40, 400
+    K, V, e = cases.synthetic_unit(9, 1, 0, 0, L0 + steps)
+    Q = cases.synthetic_queries(9, 1, 0, 0, G, steps)
+    u = OracleUnit(G=G, k_q=k_q, k_e=k_e, cap=4096, fill=True)
+    u.prefill(K[:L0], V[:L0], e[:L0])
+    dropped = set()
+    shrank = 0
+    for t in range(steps):
+        r = u.step(K[L0 + t], V[L0 + t], float(e[L0 + t]), Q[t])
+        E = u.E()
+        nb_c = (u.length - 1) // 64
+        gq, ge = set(r["gq"].tolist()), set(r["ge"].tolist())
+        assert not (gq & ge)
+        assert not (ge & dropped), t
+        elig = [b for b in range(nb_c) if b not in gq and b not in dropped]
+        assert len(ge) == min(k_e, len(elig))
+        shrank += len(gq) + len(ge) < k_q + k_e
+        worst = min(ge, key=lambda b: (E[b], -b)) if ge else None
+        for b in elig:
+            if b not in ge:
+                assert (E[b], -b) < (E[worst], -worst), (t, b, worst)
+        sel = set(r["sel"].tolist())
+        dropped |= {b for b in range(nb_c) if b not in sel}
+    v = u.violations()
+    assert v["gamma"] == 0 and v["reselect"] == 0 and v["fetch"] == 0
+    assert shrank > 0  # the case where Gamma_q takes eligible blocks and Sel holds fewer than k
+
+
+def test_bf16_pooled_keys_barely_move_the_selection():
+    """bf16 rounding of the pooled keys moves few Gamma_q blocks on the synthetic workload (a bound on
+    how far the bf16 variant departs from fp32 storage, not a pin of either)."""
+    swapped = total = 0
+    L0, steps = 8192, 24
+    for unit in range(2):
+        K, V, e = cases.synthetic_unit(0, 0, unit, 0, L0 + steps)
+        Q = cases.synthetic_queries(0, 0, unit, 0, 8, steps)
+        a = OracleUnit(G=8, k_q=16, k_e=48, cap=16384)
+        b = OracleUnit(G=8, k_q=16, k_e=48, cap=16384, ck_bf16=True)
+        a.prefill(K[:L0], V[:L0], e[:L0])
+        b.prefill(K[:L0], V[:L0], e[:L0])
+        for t in range(steps):
+            ra = a.step(K[L0 + t], V[L0 + t], float(e[L0 + t]), Q[t])
+            rb = b.step(K[L0 + t], V[L0 + t], float(e[L0 + t]), Q[t])
+            swapped += len(set(ra["gq"].tolist()) - set(rb["gq"].tolist()))
+            total += len(ra["gq"])
+    assert swapped <= 0.01 * total, (swapped, total)
