@@ -59,6 +59,8 @@ def describe(c, groups):
         s += "KV resident in device memory"
     if c.get("ck_bf16"):
         s += ", pooled keys stored bf16"
+    if c.get("fill"):
+        s += ", fill reading of the selection"
     return s
 
 
@@ -95,7 +97,7 @@ class Workload:
         self.n_steps = n_steps
         self.max_ctx = (c["L"] + n_steps + 63) // 64 * 64
         self.cfg = nosa.make_config(self.Bm, self.Hq, self.Hkv, c["k_q"], c["k_e"], self.max_ctx, c["offload"],
-                                    ck_bf16=c.get("ck_bf16", False))
+                                    ck_bf16=c.get("ck_bf16", False), fill=c.get("fill", False))
         dev = torch.device(device)
         self.host = {}
         if c["offload"]:
@@ -435,7 +437,8 @@ def oracle_sample(c, groups, seed, n_units, n_steps, budget_s=25.0):
         V = synth.kv_rows(seed, synth.V_STREAM, kl, b, g, 0, L0 + n_steps)
         E = synth.e_rows(seed, l, b, g, 0, L0 + n_steps)
         Q = np.stack([synth.q_steps(seed, l, b, g * G + h, n_steps)[1] for h in range(G)], axis=1)
-        u = oracle.OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=cap, ck_bf16=c.get("ck_bf16", False))
+        u = oracle.OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=cap, ck_bf16=c.get("ck_bf16", False),
+                              fill=c.get("fill", False))
         u.prefill(K[:L0], V[:L0], E[:L0])
         for t in range(n_steps):
             t0 = time.perf_counter()
@@ -647,7 +650,8 @@ def run_nosa(args, c, rank, world, dev):
         "data": "synthetic (seeded counter-based generator: K,V ~ N(0,1)/sqrt(128) bf16, e ~ N(0,1), drifting q)",
         "config": {"workload": f"{args.workload}: " + describe(c, args.host_groups), "layers": c["layers"],
                    "batch": c["B"], "heads_q": c["Hq"], "heads_kv": c["Hkv"], "context": c["L"], "k_q": c["k_q"],
-                   "k_e": c["k_e"], "offload": c["offload"], "pooled_keys": "bf16" if c.get("ck_bf16") else "fp32", "host_kv_groups": args.host_groups if c["offload"] else None,
+                   "k_e": c["k_e"], "offload": c["offload"], "pooled_keys": "bf16" if c.get("ck_bf16") else "fp32",
+                   "selection": "fill" if c.get("fill") else "union", "host_kv_groups": args.host_groups if c["offload"] else None,
                    "cuda_graph": graph is not None, "micro_batches": wl.micro,
                    "l2": ("L2 flushed (256 MB write) before every timed step; steps timed one by one" if small else
                           f"inputs larger than L2: each step streams {step_bytes(wl) / 1e9:.2f} GB of pooled keys and KV blocks"),
@@ -692,6 +696,56 @@ def run_sweep(args, dev):
                                       "device_errors": errs}), flush=True)
 
 
+KQ_SWEEP = dict(k=(64, 128), kq_over_k=(0.0, 0.125, 0.25, 0.375, 0.5))
+
+
+def run_kq_sweep(args, dev):
+    """The k_q/k trade-off (montaan.com summary of 2510.13602, "Tunability": a lower k_q/k raises the
+    locality floor k_e/k): one JSON line per (k, k_q, reading) with the measured locality gamma(t),
+    the misses fetched per unit and step, |Sel| and the decode throughput.  1 layer, batch 64,
+    16 q / 2 kv heads, 128K context, KV in pinned host memory, two micro-batches; k_q <= 32."""
+    warmup, steps, stat_steps = args.warmup, args.steps, 16
+    for k in KQ_SWEEP["k"]:
+        for frac in KQ_SWEEP["kq_over_k"]:
+            kq = int(round(frac * k))
+            if kq > 32:
+                continue
+            for fill in (False, True):
+                c = dict(layers=1, B=64, Hq=16, Hkv=2, L=131072, k_q=kq, k_e=k - kq, offload=True, fill=fill,
+                         ck_bf16=args.ck_bf16)
+                wl = Workload(c, stat_steps + warmup + steps + 1, seed=args.seed, device=dev, micro=2)
+                prev, gam, miss, nsel = None, [], [], []
+                for t in range(stat_steps):
+                    wl.cur.copy_(wl.inputs[t])
+                    wl.launch_step()
+                    torch.cuda.synchronize()
+                    now = [(lay.sel.cpu().numpy(), lay.nsel.cpu().numpy(), lay.n_fetched.cpu().numpy())
+                           for lay in wl.layers[0]]
+                    for m, (sel, ns, nf) in enumerate(now):
+                        for u in range(sel.shape[0]):
+                            cur = set(sel[u, :ns[u] - 1].tolist())  # Sel(t): S(t) without the local block
+                            nsel.append(len(cur))
+                            if t > 0:
+                                miss.append(int(nf[u]))
+                            if prev is not None and cur:
+                                before = set(prev[m][0][u, :prev[m][1][u]].tolist())
+                                gam.append(len(cur & before) / len(cur))
+                    prev = now
+                ms, _ = wl.time_steps(warmup, steps, first=stat_steps)
+                errs = [lay.read_error() for per in wl.layers for lay in per]
+                del wl
+                torch.cuda.empty_cache()
+                print(json.dumps({"kq_sweep": {"k": k, "k_q": kq, "k_e": k - kq, "kq_over_k": kq / k,
+                                               "selection": "fill" if fill else "union",
+                                               "pooled_keys": "bf16" if args.ck_bf16 else "fp32"},
+                                  "gamma_mean": float(np.mean(gam)), "gamma_min": float(np.min(gam)),
+                                  "gamma_floor": (k - kq) / k, "misses_per_unit_step": float(np.mean(miss)),
+                                  "sel_per_unit": float(np.mean(nsel)),
+                                  "tokens_per_s": c["B"] / (ms * 1e-3), "ms_per_step": ms,
+                                  "stat_steps": stat_steps, "steps": steps, "warmup": warmup,
+                                  "device_errors": errs}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -711,10 +765,16 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="batch x context x k sweep against dense decode (one JSON line per point)")
     ap.add_argument("--ck-bf16", action="store_true", help="store pooled keys as bf16 instead of fp32")
+    ap.add_argument("--kq-sweep", action="store_true",
+                    help="gamma, misses and throughput against k_q/k, union and fill (one JSON line per point)")
+    ap.add_argument("--fill", action="store_true",
+                    help="fill reading of the selection: Gamma_e fills the remainder outside Gamma_q")
     args = ap.parse_args()
     c = dict(WORKLOADS[args.workload])
     if args.ck_bf16:
         c["ck_bf16"] = True
+    if args.fill:
+        c["fill"] = True
     if args.layers is not None:
         c["layers"] = args.layers
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -732,6 +792,9 @@ def main():
     nosa.lib()
     if args.sweep:
         run_sweep(args, dev)
+        return
+    if args.kq_sweep:
+        run_kq_sweep(args, dev)
         return
     try:
         run_nosa(args, c, rank, world, dev)

@@ -26,9 +26,9 @@ NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", 
 
 OK, ERR_ARG, ERR_CAPACITY, ERR_PTR, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED, ERR_DEVICE = 0, -1, -2, -3, -4, -5, -6, -7
 EFLAG_CAPACITY, EFLAG_TIMEOUT, EFLAG_NOSLOT, EFLAG_STATE = 1, 2, 4, 8
-FLAG_CK_BF16 = 1
+FLAG_CK_BF16, FLAG_FILL = 1, 2
 (BUF_KV_STORE, BUF_EVICT_LOGIT, BUF_CK, BUF_BLK_EVICT, BUF_GAMMA_E, BUF_GAMMA_N, BUF_SEQ_LEN, BUF_CACHE,
- BUF_SLOT_BLOCK, BUF_BLOCK_SLOT, BUF_ERR) = range(11)
+ BUF_SLOT_BLOCK, BUF_BLOCK_SLOT, BUF_ERR, BUF_POOL, BUF_POOL_N) = range(13)
 WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC = 0, 1, 2, 3
 
 # Every extern "C" symbol include/nosa.h declares.
@@ -63,7 +63,8 @@ class Config(ctypes.Structure):
 
 class State(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ["kv_store", "evict_logit", "ck", "blk_evict", "gamma_e", "gamma_n",
-                                              "seq_len", "cache", "slot_block", "block_slot", "err"]]
+                                              "seq_len", "cache", "slot_block", "block_slot", "err", "pool",
+                                              "pool_n"]]
 
 
 _lib = None
@@ -118,10 +119,10 @@ def _stream(stream):
 
 
 def make_config(batch, heads_q, heads_kv, k_q, k_e, max_ctx, offload=False, head_dim=128, block=64, sub_block=16,
-                scale=None, ck_bf16=False):
+                scale=None, ck_bf16=False, fill=False):
     return Config(batch, heads_q, heads_kv, head_dim, block, sub_block, k_q, k_e, 1, int(bool(offload)),
                   int(max_ctx), float(scale if scale is not None else head_dim ** -0.5),
-                  FLAG_CK_BF16 if ck_bf16 else 0)
+                  (FLAG_CK_BF16 if ck_bf16 else 0) | (FLAG_FILL if fill else 0))
 
 
 # ---- the C entry points, one to one -------------------------------------------------
@@ -229,9 +230,11 @@ class NosaLayer:
         self.slot_block = dbuf(BUF_SLOT_BLOCK, torch.int32)
         self.block_slot = dbuf(BUF_BLOCK_SLOT, torch.int32)
         self.err = dbuf(BUF_ERR, torch.int32)
+        self.pool = dbuf(BUF_POOL, torch.int32)
+        self.pool_n = dbuf(BUF_POOL_N, torch.int32)
         self.state = State(*[None if t is None else t.data_ptr() for t in (
             self.kv_store, self.evict_logit, self.ck, self.blk_evict, self.gamma_e, self.gamma_n, self.seq_len,
-            self.cache, self.slot_block, self.block_slot, self.err)])
+            self.cache, self.slot_block, self.block_slot, self.err, self.pool, self.pool_n)])
         # per-step outputs and workspaces (zero-filled once, as the library requires)
         self.sel = torch.full((self.units, self.max_sel), -1, dtype=torch.int32, device=dev)
         self.nsel = torch.zeros(self.units, dtype=torch.int32, device=dev)

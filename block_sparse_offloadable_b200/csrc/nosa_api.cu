@@ -81,6 +81,9 @@ int check_state(const nosa_config *c, const nosa_state *st) {
             (rc = check_dev(st->block_slot, false)))
             return rc;
     }
+    if ((c->flags & NOSA_FLAG_FILL) &&
+        ((rc = check_dev(st->pool, false)) || (rc = check_dev(st->pool_n, false))))
+        return rc;
     return NOSA_OK;
 }
 
@@ -200,7 +203,7 @@ int nosa_validate_config(const nosa_config *c) {
     if (!c) return NOSA_ERR_ARG;
     if (c->batch < 1 || c->heads_kv < 1 || c->heads_q < 1 || c->heads_q % c->heads_kv) return NOSA_ERR_ARG;
     if (c->k_q < 0 || c->k_e < 0 || c->k_q + c->k_e < 1 || c->max_ctx <= 0 ||
-        c->max_ctx % 64 || (c->flags & ~NOSA_FLAG_CK_BF16) != 0 || !(c->scale > 0.f) || !isfinite(c->scale))
+        c->max_ctx % 64 || (c->flags & ~(NOSA_FLAG_CK_BF16 | NOSA_FLAG_FILL)) != 0 || !(c->scale > 0.f) || !isfinite(c->scale))
         return NOSA_ERR_ARG;
     if (c->offload != 0 && c->offload != 1) return NOSA_ERR_ARG;
     if (c->head_dim != kD || c->block != kBlock || c->sub_block != kSub || c->local_blocks != 1)
@@ -231,6 +234,8 @@ size_t nosa_state_bytes(const nosa_config *c, int which) {
     case NOSA_BUF_SLOT_BLOCK: return c->offload ? u * g.nslots * sizeof(int32_t) : 0;
     case NOSA_BUF_BLOCK_SLOT: return c->offload ? u * g.nblk * sizeof(int32_t) : 0;
     case NOSA_BUF_ERR: return sizeof(uint32_t);
+    case NOSA_BUF_POOL: return (c->flags & NOSA_FLAG_FILL) ? u * g.nblk * sizeof(int32_t) : 0;
+    case NOSA_BUF_POOL_N: return (c->flags & NOSA_FLAG_FILL) ? u * sizeof(int32_t) : 0;
     default: return 0;
     }
 }
@@ -247,6 +252,8 @@ int nosa_state_init(const nosa_config *c, const nosa_state *st, void *stream) {
     bool ok = cudaMemsetAsync(st->gamma_n, 0, nosa_state_bytes(c, NOSA_BUF_GAMMA_N), cs) == cudaSuccess &&
               cudaMemsetAsync(st->seq_len, 0, nosa_state_bytes(c, NOSA_BUF_SEQ_LEN), cs) == cudaSuccess &&
               cudaMemsetAsync(st->err, 0, sizeof(uint32_t), cs) == cudaSuccess;
+    if (ok && (c->flags & NOSA_FLAG_FILL))
+        ok = cudaMemsetAsync(st->pool_n, 0, nosa_state_bytes(c, NOSA_BUF_POOL_N), cs) == cudaSuccess;
     if (ok && c->offload) {
         ok = cudaMemsetAsync(st->slot_block, 0xFF, nosa_state_bytes(c, NOSA_BUF_SLOT_BLOCK), cs) == cudaSuccess &&
              cudaMemsetAsync(st->block_slot, 0xFF, nosa_state_bytes(c, NOSA_BUF_BLOCK_SLOT), cs) == cudaSuccess &&
@@ -285,6 +292,8 @@ int nosa_compress_append(const nosa_config *c, const nosa_state *st, const uint1
     p.nblk = (int32_t)g.nblk; p.nsub = (int32_t)g.nsub; p.nslots = (int32_t)g.nslots;
     p.units = (int32_t)g.units; p.heads_kv = c->heads_kv; p.k_e = c->k_e;
     p.offload = c->offload; p.T = T; p.ck_bf16 = (c->flags & NOSA_FLAG_CK_BF16) != 0;
+    p.fill = (c->flags & NOSA_FLAG_FILL) != 0;
+    p.pool = p.fill ? st->pool : nullptr; p.pool_n = p.fill ? st->pool_n : nullptr;
     return launch_append(p, static_cast<cudaStream_t>(stream));
 }
 
@@ -308,6 +317,9 @@ int nosa_select(const nosa_config *c, const nosa_state *st, const uint16_t *q, i
     p.chunk_blocks = c->k_q > 0 ? select_chunk_blocks(p.units, p.nblk, (c->flags & NOSA_FLAG_CK_BF16) != 0) : p.nblk;
     p.k_q = c->k_q; p.k_e = c->k_e; p.max_sel = (int32_t)g.max_sel; p.scale = c->scale;
     p.ck_bf16 = (c->flags & NOSA_FLAG_CK_BF16) != 0;
+    p.fill = (c->flags & NOSA_FLAG_FILL) != 0;
+    p.pool = p.fill ? st->pool : nullptr; p.pool_n = p.fill ? st->pool_n : nullptr;
+    p.gamma_e_out = p.fill ? st->gamma_e : nullptr; p.gamma_n_out = p.fill ? st->gamma_n : nullptr;
     if (p.nchunks > 1) {
         p.counter = static_cast<int32_t *>(ws);
         p.part_keys = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(ws) +

@@ -137,8 +137,35 @@ __global__ void __launch_bounds__(128) append_decode_kernel(const AppendParams p
         if (lane == 0) p.blk_evict[(int64_t)u * p.nblk + blk] = m;
     }
 
+    // fill reading: the new candidate joins the pool at its rank (E descending;
+    // it has the highest id, so it goes after every member with an equal E)
+    if (p.fill && w == 0 && blk >= 1 && p.k_e > 0) {
+        const int32_t c = blk - 1;
+        int32_t *pool = p.pool + (int64_t)u * p.nblk;
+        const double *E = p.blk_evict + (int64_t)u * p.nblk;
+        const int32_t n = p.pool_n[u];
+        const double Ec = E[c];
+        int32_t at = 0;
+        for (int i0 = 0; i0 < n; i0 += 32) {
+            const int i = i0 + lane;
+            at += __popc(__ballot_sync(0xFFFFFFFFu, i < n && E[pool[i]] >= Ec));
+        }
+        // shift [at, n) up by one, highest chunk first; each chunk is read before it is written
+        for (int top = n; top > at; top -= 32) {
+            const int i = top - 1 - lane;
+            const int32_t v = (i >= at) ? pool[i] : 0;
+            __syncwarp();
+            if (i >= at) pool[i + 1] = v;
+            __syncwarp();
+        }
+        if (lane == 0) {
+            pool[at] = c;
+            p.pool_n[u] = n + 1;
+        }
+    }
+
     // the previous local block just became a candidate: offer it to Gamma_e
-    if (w == 0 && blk >= 1 && p.k_e > 0) {
+    if (!p.fill && w == 0 && blk >= 1 && p.k_e > 0) {
         const int32_t c = blk - 1;
         int32_t *ge = p.gamma_e + (int64_t)u * p.k_e;
         const double *E = p.blk_evict + (int64_t)u * p.nblk;
@@ -241,8 +268,10 @@ __global__ void __launch_bounds__(256) prefill_pool_kernel(const AppendParams p)
     }
 }
 
-// Gamma_e := top-k_e of the candidates by E (ties to the lower block), ascending.
-// One CTA per unit; rank counting over the candidates held in shared memory.
+// Gamma_e := top-k_e of the candidates by E (ties to the lower block), ascending;
+// fill reading: also the pool of every candidate in rank order (nothing is
+// dropped before the first decode step).  One CTA per unit; rank counting over
+// the candidates held in shared memory (the ranks are a permutation).
 __global__ void __launch_bounds__(256) prefill_gamma_kernel(const AppendParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int32_t u = blockIdx.x;
@@ -256,15 +285,19 @@ __global__ void __launch_bounds__(256) prefill_gamma_kernel(const AppendParams p
     uint8_t *flag = smem + (size_t)p.nblk * sizeof(double);
     for (int i = threadIdx.x; i < nb_c; i += blockDim.x) E[i] = p.blk_evict[(int64_t)u * p.nblk + i];
     __syncthreads();
+    const bool pool = p.fill && p.k_e > 0;
+    const int32_t stop = pool ? nb_c : p.k_e;
     for (int i = threadIdx.x; i < nb_c; i += blockDim.x) {
         const double ei = E[i];
         int32_t rank = 0;
-        for (int j = 0; j < nb_c && rank < p.k_e; ++j) {
+        for (int j = 0; j < nb_c && rank < stop; ++j) {
             const double ej = E[j];
             rank += (ej > ei) || (ej == ei && j < i);
         }
         flag[i] = rank < p.k_e;
+        if (pool) p.pool[(int64_t)u * p.nblk + rank] = i;
     }
+    if (pool && threadIdx.x == 0) p.pool_n[u] = nb_c;
     __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;

@@ -23,7 +23,9 @@ struct AppendParams {
     int32_t *block_slot;     // [u][nblk]
     uint32_t *err;
     int64_t max_ctx;
-    int32_t nblk, nsub, nslots, units, heads_kv, k_e, offload, T, ck_bf16;
+    int32_t *pool;           // [u][nblk] fill reading: not-dropped candidates by E rank
+    int32_t *pool_n;         // [u]
+    int32_t nblk, nsub, nslots, units, heads_kv, k_e, offload, T, ck_bf16, fill;
 };
 
 struct SelectParams {
@@ -38,7 +40,11 @@ struct SelectParams {
     uint64_t *part_keys;      // [u][nchunks][32]
     int32_t *counter;         // [u]
     uint32_t *err;
-    int32_t nsub, nblk, G, units, nchunks, chunk_blocks, k_q, k_e, max_sel, ck_bf16;
+    int32_t *gamma_e_out;     // fill reading: Gamma_e and |Gamma_e| written here
+    int32_t *gamma_n_out;
+    int32_t *pool;            // [u][nblk] fill reading
+    int32_t *pool_n;          // [u]
+    int32_t nsub, nblk, G, units, nchunks, chunk_blocks, k_q, k_e, max_sel, ck_bf16, fill;
     float scale;
 };
 

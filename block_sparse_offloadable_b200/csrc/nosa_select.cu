@@ -67,6 +67,48 @@ __device__ __forceinline__ void reduce_level(float (&v)[32], int lane, int o) {
     }
 }
 
+// Fill reading, one warp: Gamma_e = the first k_e pool entries (E rank order)
+// outside Gamma_q, whose bits are already set in `bitmap`; their bits are set
+// too, then the pool keeps only the entries in Sel = Gamma_q + Gamma_e, in
+// order.  pf_n / pf_id: pool_n[u] and pool[u][lane], loaded early by this warp.
+__device__ __forceinline__ void fill_gamma_e(const SelectParams &p, int32_t u, int32_t nb_c, uint32_t *bitmap,
+                                             int lane, int32_t pf_n, int32_t pf_id) {
+    int32_t *pool = p.pool + (int64_t)u * p.nblk;
+    const int32_t n = pf_n;
+    int32_t *ge = p.gamma_e_out + (int64_t)u * p.k_e;
+    const unsigned lt = (1u << lane) - 1u;
+    int32_t taken = 0;
+    bool bad = false;
+    for (int i0 = 0; i0 < n && taken < p.k_e; i0 += 32) {
+        const int i = i0 + lane;
+        const int32_t id = (i < n) ? (i0 == 0 ? pf_id : pool[i]) : -1;
+        const bool ok = id >= 0 && id < nb_c;
+        bad |= (i < n) && !ok;
+        const bool elig = ok && !((bitmap[id >> 5] >> (id & 31)) & 1u);
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, elig);
+        const int32_t r = taken + __popc(m & lt);
+        if (elig && r < p.k_e) {
+            ge[r] = id;
+            atomicOr(&bitmap[id >> 5], 1u << (id & 31));
+        }
+        taken = min(taken + __popc(m), p.k_e);
+        __syncwarp();
+    }
+    if (lane == 0) p.gamma_n_out[u] = taken;
+    int32_t kept = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        const int32_t id = (i < n) ? (i0 == 0 ? pf_id : pool[i]) : -1;
+        const bool keep = id >= 0 && id < nb_c && ((bitmap[id >> 5] >> (id & 31)) & 1u);
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, keep);
+        __syncwarp();  // the chunk is read before any lane writes (writes land at or below it)
+        if (keep) pool[kept + __popc(m & lt)] = id;
+        kept += __popc(m);
+    }
+    if (lane == 0) p.pool_n[u] = kept;
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_error(p.err, NOSA_EFLAG_STATE);
+}
+
 template <typename T>
 size_t select_smem_bytes(int32_t nblk) {
     constexpr int S = SelGeo<T>::kStages;
@@ -117,8 +159,14 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
     }
     __syncthreads();
 
-    // warp 0 may finalize this unit: fetch Gamma_e now, while the stream runs
-    const int32_t ne = (warp == 0) ? min(p.gamma_n[u], p.k_e) : 0;
+    // warp 0 may finalize this unit: fetch Gamma_e (fill reading: the head of
+    // the pool) now, while the stream runs
+    const int32_t ne = (warp == 0 && !p.fill) ? min(p.gamma_n[u], p.k_e) : 0;
+    int32_t pf_n = 0, pf_id = -1;
+    if (warp == 0 && p.fill) {
+        pf_n = min(max(p.pool_n[u], 0), p.nblk);  // a pool never holds more than nblk - 1 ids
+        if (lane < pf_n) pf_id = p.pool[(int64_t)u * p.nblk + lane];
+    }
     int32_t ge_reg[kMaxKe / 32];
     if (warp == 0) {
         const int32_t *ge = p.gamma_e + (int64_t)u * p.k_e;
@@ -229,7 +277,10 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
     int32_t *sel = p.sel + (int64_t)u * p.max_sel;
     if (L <= 0) {
         for (int i = lane; i < p.max_sel; i += 32) sel[i] = -1;
-        if (lane == 0) p.nsel[u] = 0;
+        if (lane == 0) {
+            p.nsel[u] = 0;
+            if (p.fill) p.gamma_n_out[u] = 0;
+        }
         return;
     }
     const int32_t nw = (nb_c + 31) >> 5;
@@ -242,6 +293,10 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
         if (id >= 0 && id < nb_c) atomicOr(&bitmap[id >> 5], 1u << (id & 31));
     }
     __syncwarp();
+    if (p.fill) {
+        fill_gamma_e(p, u, nb_c, bitmap, lane, pf_n, pf_id);
+        __syncwarp();
+    }
     const int32_t per = (nw + 31) / 32;
     const int32_t w0 = min(lane * per, nw), w1 = min(w0 + per, nw);
     int32_t cnt = 0;

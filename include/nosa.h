@@ -87,6 +87,18 @@ typedef struct nosa_config {
 #define NOSA_FLAG_CK_BF16 0x1
 
 /*
+ * "Fill" combination of the two selections (montaan.com summary of
+ * 2510.13602, "Key Design Components" item 4: query-aware blocks first, the
+ * remainder filled with query-agnostic ones; item 1: a block the selection
+ * lets go is never selected by the query-agnostic part again).  Gamma_e is
+ * then the top-k_e by E among the candidates outside Gamma_q that have been
+ * selected at every step since they became candidates (or since the
+ * prefill); Sel = Gamma_q and Gamma_e are disjoint, |Sel| <= k.  Without the
+ * flag Gamma_e is the independent top-k_e and Sel their union.
+ */
+#define NOSA_FLAG_FILL 0x2
+
+/*
  * Per-layer state.  Every buffer is caller-owned; nosa_state_bytes(cfg, NOSA_BUF_x)
  * gives its size.  Layouts (u = unit, nblk = max_ctx/64, nsub = max_ctx/16,
  * nslots = k_q + k_e + 2):
@@ -103,6 +115,9 @@ typedef struct nosa_config {
  *   slot_block  int32 [u][nslots]   block held by each cache slot, -1 = free (device; offload only)
  *   block_slot  int32 [u][nblk]     cache slot of each block, -1 = not resident (device; offload only)
  *   err         uint32 [1]          device error word (device)
+ *   pool        int32 [u][nblk]     NOSA_FLAG_FILL only: the candidates not yet dropped,
+ *               sorted by E descending, ties to the lower block (device; NULL otherwise)
+ *   pool_n      int32 [u]           NOSA_FLAG_FILL only: entries in pool (device)
  * nosa_state_init must run once before the first append.
  */
 typedef struct nosa_state {
@@ -117,6 +132,8 @@ typedef struct nosa_state {
     int32_t *slot_block;
     int32_t *block_slot;
     uint32_t *err;
+    int32_t *pool;
+    int32_t *pool_n;
 } nosa_state;
 
 enum nosa_buffer {
@@ -131,6 +148,8 @@ enum nosa_buffer {
     NOSA_BUF_SLOT_BLOCK,
     NOSA_BUF_BLOCK_SLOT,
     NOSA_BUF_ERR,
+    NOSA_BUF_POOL,
+    NOSA_BUF_POOL_N,
     NOSA_BUF_COUNT
 };
 
@@ -179,8 +198,11 @@ int nosa_state_init(const nosa_config *cfg, const nosa_state *st, void *stream);
  * its sub-blocks of the mean eviction logit (fp64); when a block becomes a
  * candidate, it enters Gamma_e if |Gamma_e| < k_e, or replaces the member with
  * the lowest E if its E is strictly higher (the member is then dropped for
- * good).  Prefill builds the pooled arrays and Gamma_e = top-k_e by E (ties
- * to the lower block) and, in offload mode, puts the local block in the cache.
+ * good).  With NOSA_FLAG_FILL the candidate instead joins the pool at its
+ * rank, and nosa_select forms Gamma_e.  Prefill builds the pooled arrays and
+ * Gamma_e = top-k_e by E (ties to the lower block), with NOSA_FLAG_FILL the
+ * pool of every candidate in rank order, and, in offload mode, puts the local
+ * block in the cache.
  * Device errors: NOSA_EFLAG_CAPACITY (L + T > max_ctx; unit skipped),
  * NOSA_EFLAG_STATE (prefill into a non-empty unit), NOSA_EFLAG_NOSLOT.
  */
@@ -205,7 +227,9 @@ int nosa_compress_append(const nosa_config *cfg, const nosa_state *st, const uin
  * s_b = max over the four sub-blocks s of b of  (sum over the G query heads h
  * of kv head g of q_h) . kbar_s * scale, in fp32, for every candidate b;
  * Gamma_q = the k_q highest (ties to the lower block).  Uses Gamma_e as left
- * by nosa_compress_append.
+ * by nosa_compress_append; with NOSA_FLAG_FILL, takes Gamma_e = the first
+ * k_e pool entries outside Gamma_q (written to gamma_e in rank order, and
+ * gamma_n), then keeps in the pool only the entries in Sel.
  */
 int nosa_select(const nosa_config *cfg, const nosa_state *st, const uint16_t *q, int32_t *sel,
                 int32_t *nsel, int32_t *gq, void *ws, size_t ws_bytes, void *stream);

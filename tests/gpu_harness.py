@@ -8,7 +8,11 @@ inputs, and compare them with the tolerances the library is held to:
 * outputs (bf16) within max-abs 1e-2 and mean-abs 1e-3 of the fp64 oracle, and,
   tighter, a relative L2 error <= 1e-2 (bf16 rounding of P and of the output
   gives ~3e-3);
-* offload fetch counts bit-exact while the unit's selection history matches.
+* offload fetch counts bit-exact while the unit's selection history matches;
+* fill reading: Gamma_e depends on Gamma_q and on the drop history, so after an
+  excused near-tie the unit's later selections are only checked for being
+  self-consistent (Gamma_e disjoint from Gamma_q, S(t) their union plus the
+  local block) and counted as `diverged`.
 """
 import numpy as np
 import torch
@@ -23,7 +27,7 @@ MAX_ABS, MEAN_ABS, REL_L2 = 1e-2, 1e-3, 1e-2
 
 class Scenario:
     def __init__(self, B, Hq, Hkv, k_q, k_e, L0, steps, offload=False, seed=0, layer=0, lens=None,
-                 max_ctx=None, dense=False, ck_bf16=False):
+                 max_ctx=None, dense=False, ck_bf16=False, fill=False):
         self.B, self.Hq, self.Hkv, self.k_q, self.k_e = B, Hq, Hkv, k_q, k_e
         self.G = Hq // Hkv
         self.units = B * Hkv
@@ -33,10 +37,11 @@ class Scenario:
         self.max_ctx = max_ctx or ((self.Lmax + 63) // 64 * 64 + 64)
         self.dense = dense
         self.ck_bf16 = ck_bf16
+        self.fill = fill
 
     def cfg(self):
         return nosa.make_config(self.B, self.Hq, self.Hkv, self.k_q, self.k_e, self.max_ctx, self.offload,
-                                ck_bf16=self.ck_bf16)
+                                ck_bf16=self.ck_bf16, fill=self.fill)
 
 
 def unit_data(sc):
@@ -113,38 +118,47 @@ def _tie_ok(sa, sb, smax):
 
 
 def new_stats():
-    return dict(cmp=0, exact=0, excused=0, unexcused=0, ge_mismatch=0, fetch_cmp=0, fetch_mismatch=0,
+    return dict(cmp=0, exact=0, excused=0, diverged=0, unexcused=0, ge_mismatch=0, fetch_cmp=0, fetch_mismatch=0,
                 max_abs=0.0, sum_abs=0.0, n_out=0, max_rel=0.0, dense_max_abs=0.0, dense_max_rel=0.0,
                 gamma_min=1.0)
 
 
-def compare_step(st, o, r, q, gsel, ggq, gge, gout, k_q, history_ok, gfetch=None, report=None, tag=None):
+def compare_step(st, o, r, q, gsel, ggq, gge, gout, k_q, history_ok, gfetch=None, report=None, tag=None,
+                 fill=False):
     """Compare one (unit, step) of the GPU path with the oracle's step result r.
 
     gsel: GPU S(t) (ascending, local last); ggq: GPU Gamma_q ids (rank order, -1 padded);
     gge: GPU Gamma_e ids (any order) or None; gout: GPU output [G][D] as float.
     Returns the updated history flag (False once the selections have differed)."""
     st["cmp"] += 1
-    if gge is not None and not np.array_equal(np.sort(gge), r["ge"]):
+    gq_set = set(x for x in list(ggq)[:k_q] if x >= 0)
+    oq_set = set(r["gq"].tolist())
+    ge_set = set(gge.tolist()) if gge is not None else set()
+    if gge is not None and (not fill or (history_ok and gq_set == oq_set)) and not np.array_equal(np.sort(gge), r["ge"]):
         st["ge_mismatch"] += 1
     if np.array_equal(gsel, r["sel"]):
         st["exact"] += 1
         ref = r["o"]
     else:
-        history_ok = False
-        gq_set = set(x for x in list(ggq)[:k_q] if x >= 0)
-        oq_set = set(r["gq"].tolist())
         s = r["scores"]
         smax = float(np.abs(s).max()) if len(s) else 0.0
         a = sorted(gq_set - oq_set, key=lambda x: -s[x])
         bb = sorted(oq_set - gq_set, key=lambda x: -s[x])
-        consistent = np.array_equal(gsel, np.array(sorted(gq_set | set(r["ge"].tolist())) + [r["local"]]))
-        if consistent and len(a) == len(bb) and all(_tie_ok(s[x], s[y], smax) for x, y in zip(a, bb)):
+        if fill:
+            consistent = (not (gq_set & ge_set) and
+                          np.array_equal(gsel, np.array(sorted(gq_set | ge_set) + [r["local"]])))
+        else:
+            consistent = np.array_equal(gsel, np.array(sorted(gq_set | set(r["ge"].tolist())) + [r["local"]]))
+        ties = len(a) == len(bb) and all(_tie_ok(s[x], s[y], smax) for x, y in zip(a, bb))
+        if fill and not history_ok and consistent:
+            st["diverged"] += 1
+        elif consistent and ties:
             st["excused"] += 1
         else:
             st["unexcused"] += 1
             if report is not None:
                 report.append((tag, list(gsel), r["sel"].tolist()))
+        history_ok = False
         ref = o.attend_blocks(q, gsel)
     err = np.abs(gout - ref)
     st["max_abs"] = max(st["max_abs"], float(err.max()))
@@ -168,7 +182,7 @@ def compare(sc, data, gpu, units=None, report=None):
     for u in units:
         b, g = divmod(u, sc.Hkv)
         n0 = sc.lens[b]
-        o = OracleUnit(G=sc.G, k_q=sc.k_q, k_e=sc.k_e, cap=sc.max_ctx, ck_bf16=sc.ck_bf16)
+        o = OracleUnit(G=sc.G, k_q=sc.k_q, k_e=sc.k_e, cap=sc.max_ctx, ck_bf16=sc.ck_bf16, fill=sc.fill)
         if n0 > 0:
             o.prefill(K[u, :n0], V[u, :n0], E[u, :n0])
         history_ok = True
@@ -180,7 +194,7 @@ def compare(sc, data, gpu, units=None, report=None):
             gge = gpu["ge"][t][u][: gpu["gn"][t][u]] if sc.k_e else None
             history_ok = compare_step(st, o, r, q, gsel, gpu["gq"][t][u], gge,
                                       gpu["out"][t][b, g * sc.G:(g + 1) * sc.G], sc.k_q, history_ok,
-                                      gpu["nf"][t][u] if sc.offload else None, report, (t, u))
+                                      gpu["nf"][t][u] if sc.offload else None, report, (t, u), sc.fill)
             if sc.dense:
                 dref = o.dense(q)
                 dg = gpu["dense"][t][b, g * sc.G:(g + 1) * sc.G]

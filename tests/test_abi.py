@@ -43,8 +43,9 @@ def test_validate_config(L):
     assert nosa.nosa_validate_config(cfg(max_ctx=1 << 21)) == nosa.ERR_CAPACITY
     assert nosa.nosa_validate_config(cfg(batch=1024, max_ctx=1 << 20)) == nosa.ERR_CAPACITY
     assert nosa.nosa_validate_config(cfg(ck_bf16=True)) == nosa.OK
+    assert nosa.nosa_validate_config(cfg(ck_bf16=True, fill=True)) == nosa.OK
     bad = cfg()
-    bad.flags = 2  # an undefined flag bit
+    bad.flags = 4  # an undefined flag bit
     assert nosa.nosa_validate_config(bad) == nosa.ERR_ARG
 
 
@@ -61,6 +62,9 @@ def test_state_sizes(L):
     assert nosa.nosa_state_bytes(co, nosa.BUF_BLOCK_SLOT) == u * nblk * 4
     assert nosa.nosa_state_bytes(cfg(max_ctx=100), nosa.BUF_CK) == 0  # invalid config
     assert nosa.nosa_state_bytes(cfg(ck_bf16=True), nosa.BUF_CK) == u * (8192 // 16) * 128 * 2
+    assert nosa.nosa_state_bytes(c, nosa.BUF_POOL) == 0 and nosa.nosa_state_bytes(c, nosa.BUF_POOL_N) == 0
+    assert nosa.nosa_state_bytes(cfg(fill=True), nosa.BUF_POOL) == u * nblk * 4
+    assert nosa.nosa_state_bytes(cfg(fill=True), nosa.BUF_POOL_N) == u * 4
 
 
 def test_workspace_sizes_cover_chunks(L):

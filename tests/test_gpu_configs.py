@@ -72,14 +72,15 @@ def run_config(c, steps, seqs=None, seed=0, micro=1, dense_step=None, name=None)
         V = synth.kv_rows(seed, synth.V_STREAM, wl.kv_layer(0), b, g, 0, L0 + steps)
         E = synth.e_rows(seed, 0, b, g, 0, L0 + steps)
         Q = np.stack([synth.q_steps(seed, 0, b, g * G + h, steps)[1] for h in range(G)], axis=1)
-        o = OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=wl.max_ctx, ck_bf16=c.get("ck_bf16", False))
+        o = OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=wl.max_ctx, ck_bf16=c.get("ck_bf16", False),
+                       fill=c.get("fill", False))
         o.prefill(K[:L0], V[:L0], E[:L0])
         ok = True
         for t in range(steps):
             r = o.step(K[L0 + t], V[L0 + t], float(E[L0 + t]), Q[t])
             g_ = rec[(b, g)][t]
             ok = H.compare_step(st, o, r, Q[t], g_["sel"], g_["gq"], g_["ge"], g_["out"], c["k_q"], ok,
-                                g_["nf"], bad, (t, b, g))
+                                g_["nf"], bad, (t, b, g), c.get("fill", False))
             if dense_out is not None and t == dense_step:
                 dref = o.dense(Q[t])
                 dg = dense_out[b, g * G:(g + 1) * G]
