@@ -54,6 +54,7 @@ def lib():
         L.nosa_oracle_attend_blocks.argtypes = [P, P, P, ctypes.c_int32, P]
         L.nosa_oracle_set_ck_bf16.argtypes = [P, ctypes.c_int32]
         L.nosa_oracle_set_fill.argtypes = [P, ctypes.c_int32]
+        L.nosa_oracle_evict_head.argtypes = [P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, P, P, P]
         L.nosa_oracle_round_bf16.argtypes = [ctypes.c_double]
         L.nosa_oracle_round_bf16.restype = ctypes.c_double
         _lib = L
@@ -67,6 +68,20 @@ def _p(a):
 def round_bf16(x):
     """x rounded to the nearest bf16 value, ties to even (the oracle's rounding of pooled keys)."""
     return lib().nosa_oracle_round_bf16(float(x))
+
+
+def evict_head(V, W1, W2):
+    """Eviction logits of value rows V [T][D] (bf16 bits) under one head W1 [D][H], W2 [H] (fp32):
+    e_j = sum_h W2[h] softplus(v_j . W1[:, h]), fp64, rounded to fp32."""
+    V = np.ascontiguousarray(V, dtype=np.uint16)
+    W1 = np.ascontiguousarray(W1, dtype=np.float32)
+    W2 = np.ascontiguousarray(W2, dtype=np.float32)
+    T, D = V.shape
+    H = W2.shape[0]
+    assert W1.shape == (D, H)
+    e = np.empty(T, np.float32)
+    lib().nosa_oracle_evict_head(_p(V), T, D, H, _p(W1), _p(W2), _p(e))
+    return e
 
 
 class OracleUnit:

@@ -153,6 +153,32 @@ void nosa_oracle_set_ck_bf16(nosa_oracle_unit *u, int32_t on) { u->ck_bf16 = on 
 
 void nosa_oracle_set_fill(nosa_oracle_unit *u, int32_t on) { u->fill = on != 0; }
 
+/*
+ * Eviction head (montaan.com summary of 2510.13602, "Key Design Components"
+ * item 3, Equation 4; the nonlinearity is softplus, as in DMA's design):
+ *   e_j = sum_h W2[h] * softplus( sum_d v_j[d] * W1[d][h] ),
+ * for the value rows V [T][D] (bf16 bits) of one kv head, W1 [D][H], W2 [H]
+ * (fp32 values).  fp64 throughout, sums in index order, each product and sum
+ * rounded on its own; the result is rounded once to fp32 (the logits' storage
+ * type).  softplus(x) = max(x, 0) + log1p(exp(-|x|)), which neither overflows
+ * nor loses the small values.  Reading where the pages are silent: one head per
+ * layer and kv head, with hidden size H.
+ */
+static double softplus(double x) { return (x > 0.0 ? x : 0.0) + log1p(exp(-fabs(x))); }
+
+void nosa_oracle_evict_head(const uint16_t *V, int64_t T, int32_t D, int32_t H, const float *W1,
+                            const float *W2, float *e_out) {
+    for (int64_t j = 0; j < T; ++j) {
+        double e = 0.0;
+        for (int32_t h = 0; h < H; ++h) {
+            double z = 0.0;
+            for (int32_t d = 0; d < D; ++d) z += bf16_to_double(V[j * D + d]) * (double)W1[(int64_t)d * H + h];
+            e += (double)W2[h] * softplus(z);
+        }
+        e_out[j] = (float)e;
+    }
+}
+
 /* Block eviction score: max over the block's sub-blocks of the mean eviction logit. */
 static void evict_score_block(nosa_oracle_unit *u, int64_t b) {
     int32_t per = u->block / u->sub;

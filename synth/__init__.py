@@ -45,6 +45,7 @@ def host():
         L.nosa_synth_kv_rows.argtypes = [u64, u32, u32, u32, u32, u64, i64, i32, P]
         L.nosa_synth_e_rows.argtypes = [u64, u32, u32, u32, u64, i64, P]
         L.nosa_synth_q_steps.argtypes = [u64, u32, u32, u32, i64, i32, P, P]
+        L.nosa_synth_head_weights.argtypes = [u64, u32, i32, i32, i32, P, P]
         _host = L
     return _host
 
@@ -85,6 +86,14 @@ def q_steps(seed, layer, seq, qh, n, D=128):
     b = np.empty((n, D), np.uint16)
     host().nosa_synth_q_steps(seed, layer, seq, qh, n, D, _p(f), _p(b))
     return f, b
+
+
+def head_weights(seed, layer, Hkv, D=128, H=128):
+    """Synthetic eviction-head weights of one layer: W1 fp32 [Hkv][D][H], W2 fp32 [Hkv][H]."""
+    W1 = np.empty((Hkv, D, H), np.float32)
+    W2 = np.empty((Hkv, H), np.float32)
+    host().nosa_synth_head_weights(seed, layer, Hkv, D, H, _p(W1), _p(W2))
+    return W1, W2
 
 
 def bf16_to_f32(bits):

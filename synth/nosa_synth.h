@@ -27,6 +27,10 @@
  *   e     : z (fp32).
  *   q     : q_0 = z_0, q_t = 0.9f*q_{t-1} + 0.44f*z_t, each product and the
  *           sum rounded to fp32 separately; the kernel input is bf16(q_t).
+ *   W1, W2: weights of a synthetic eviction head (random, untrained), per
+ *           layer and kv head, fp32: W1 [D][H] (row d, column h) = z, so that
+ *           v.W1 has unit variance for v ~ N(0,1)/sqrt(128); W2 [H] =
+ *           z * (1/sqrt(128)).
  */
 #ifndef NOSA_SYNTH_H
 #define NOSA_SYNTH_H
@@ -44,6 +48,8 @@
 #define NOSA_SYNTH_V 2u
 #define NOSA_SYNTH_E 3u
 #define NOSA_SYNTH_Q 4u
+#define NOSA_SYNTH_W1 5u
+#define NOSA_SYNTH_W2 6u
 
 /* 1/sqrt((2^32-1)/3): unit-variance scale for the centred 4-draw sum. */
 #define NOSA_SYNTH_C_UNIT 0x1.bb67aep-16f   /* 2.6428997e-05, fp32-exact */
@@ -111,6 +117,7 @@ NOSA_SYNTH_FN float nosa_synth_normal(uint64_t row, uint32_t dim) {
 NOSA_SYNTH_FN uint16_t nosa_synth_kv(uint64_t row, uint32_t dim) {
     return nosa_synth_bf16(nosa_synth_fmul((float)nosa_synth_centred(row, dim), NOSA_SYNTH_C_KV));
 }
+
 
 /* eviction logit of one token: N(0,1) fp32 */
 NOSA_SYNTH_FN float nosa_synth_e(uint64_t seed, uint32_t layer, uint32_t seq, uint32_t kvh,

@@ -40,3 +40,17 @@ void nosa_synth_q_steps(uint64_t seed, uint32_t layer, uint32_t seq, uint32_t qh
         }
     }
 }
+
+/* Synthetic eviction-head weights of one layer: W1 [Hkv][D][H], W2 [Hkv][H] (fp32). */
+void nosa_synth_head_weights(uint64_t seed, uint32_t layer, int32_t Hkv, int32_t D, int32_t H, float *W1,
+                             float *W2) {
+    for (int32_t g = 0; g < Hkv; ++g) {
+        for (int32_t d = 0; d < D; ++d) {
+            uint64_t row = nosa_synth_row(seed, NOSA_SYNTH_W1, layer, 0u, (uint32_t)g, (uint64_t)d);
+            for (int32_t h = 0; h < H; ++h) W1[((int64_t)g * D + d) * H + h] = nosa_synth_normal(row, (uint32_t)h);
+        }
+        uint64_t row = nosa_synth_row(seed, NOSA_SYNTH_W2, layer, 0u, (uint32_t)g, 0u);
+        for (int32_t h = 0; h < H; ++h)
+            W2[(int64_t)g * H + h] = nosa_synth_fmul((float)nosa_synth_centred(row, (uint32_t)h), NOSA_SYNTH_C_KV);
+    }
+}

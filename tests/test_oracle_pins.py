@@ -368,3 +368,73 @@ def test_bf16_pooled_keys_barely_move_the_selection():
             swapped += len(set(ra["gq"].tolist()) - set(rb["gq"].tolist()))
             total += len(ra["gq"])
     assert swapped <= 0.01 * total, (swapped, total)
+
+
+def _bf16_bits(x):
+    return (np.asarray(x, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_evict_head_zero_first_layer_gives_ln2_times_sum():
+    """W1 = 0 makes every hidden pre-activation 0 and softplus(0) = ln 2, so e = ln 2 * sum(W2)."""
+    import oracle
+    _, W2 = synth.head_weights(3, 0, 1)
+    V = synth.kv_rows(3, synth.V_STREAM, 0, 0, 0, 0, 5)
+    e = oracle.evict_head(V, np.zeros((128, 128), np.float32), W2[0])
+    want = np.float32(np.log(2.0) * np.sum(W2[0].astype(np.float64)))
+    assert np.all(np.abs(e - want) <= np.spacing(np.abs(want)))
+
+
+def test_evict_head_single_path_and_orientation():
+    """One nonzero W1 entry (row d0, column h0) and W2 = c at h0 only: e_j = c * log(1 + exp(a v_j[d0])).
+    A transposed W1 (row h0, column d0) would read a different input dimension."""
+    import oracle
+    d0, h0, a, c = 5, 77, 3.0, 0.75
+    W1 = np.zeros((128, 128), np.float32)
+    W1[d0, h0] = a
+    W2 = np.zeros(128, np.float32)
+    W2[h0] = c
+    V = synth.kv_rows(4, synth.V_STREAM, 0, 0, 0, 0, 64)
+    vf = synth.bf16_to_f32(V).astype(np.float64)
+    want = (c * np.log(1.0 + np.exp(a * vf[:, d0]))).astype(np.float32)
+    got = oracle.evict_head(V, W1, W2)
+    assert np.all(np.abs(got - want) <= np.spacing(np.abs(want)))
+    assert not np.allclose(got, (c * np.log(1.0 + np.exp(a * vf[:, h0]))).astype(np.float32))
+
+
+def test_evict_head_softplus_extremes():
+    """softplus(800) = 800 (a plain log(1+exp) overflows) and softplus(-40) = exp(-40) to within
+    1e-17 relative (a plain log(1+exp) gives 0)."""
+    import oracle
+    W1 = np.zeros((128, 128), np.float32)
+    W1[0, 0], W1[0, 1] = 800.0, -40.0
+    V = np.zeros((1, 128), np.uint16)
+    V[0, 0] = _bf16_bits(1.0)
+    for h, want in ((0, 800.0), (1, np.exp(-40.0))):
+        W2 = np.zeros(128, np.float32)
+        W2[h] = 1.0
+        got = oracle.evict_head(V, W1, W2)[0]
+        assert got == np.float32(want), (h, got, want)
+
+
+def test_evict_head_matches_numpy_logaddexp():
+    """The head on seeded inputs against NumPy's fp64 matmul and logaddexp(0, z) = softplus(z):
+    equal to within one fp32 unit in the last place (the two sum in different orders)."""
+    import oracle
+    W1, W2 = synth.head_weights(7, 2, 2)
+    V = synth.kv_rows(7, synth.V_STREAM, 2, 1, 1, 0, 300)
+    vf = synth.bf16_to_f32(V).astype(np.float64)
+    for g in range(2):
+        want = np.logaddexp(0.0, vf @ W1[g].astype(np.float64)) @ W2[g].astype(np.float64)
+        got = oracle.evict_head(V, W1[g], W2[g])
+        assert np.all(np.abs(got.astype(np.float64) - want) <= np.spacing(np.abs(want).astype(np.float32))), g
+    assert got.std() > 0.2  # the synthetic head is not degenerate
+
+
+def test_evict_head_is_linear_in_second_layer():
+    import oracle
+    W1, W2 = synth.head_weights(8, 0, 2)
+    V = synth.kv_rows(8, synth.V_STREAM, 0, 0, 0, 0, 50)
+    a = oracle.evict_head(V, W1[0], W2[0]).astype(np.float64)
+    b = oracle.evict_head(V, W1[0], W2[1]).astype(np.float64)
+    ab = oracle.evict_head(V, W1[0], W2[0] + W2[1]).astype(np.float64)
+    assert np.allclose(ab, a + b, rtol=0, atol=4e-6)
