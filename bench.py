@@ -61,6 +61,8 @@ def describe(c, groups):
         s += ", pooled keys stored bf16"
     if c.get("fill"):
         s += ", fill reading of the selection"
+    if c.get("head"):
+        s += ", eviction logits from the fused synthetic eviction head"
     return s
 
 
@@ -107,6 +109,10 @@ class Workload:
                     self.host[(g, m)] = pinned(nbytes, (g, m))
         self.layers = [[nosa.NosaLayer(self.cfg, dev, self.host[(l % groups, m)] if self.host else None)
                         for m in range(micro)] for l in range(self.L)]
+        # the fused eviction head: synthetic weights per layer (e is then computed, not an input)
+        self.head = bool(c.get("head", False))
+        self.W = [tuple(torch.from_numpy(w).to(dev) for w in synth.head_weights(seed, l, self.Hkv))
+                  for l in range(self.L)] if self.head else None
         self._prefill(dev)
         self._inputs(dev)
 
@@ -125,8 +131,11 @@ class Workload:
                 s0 = self.seq_base + m * self.Bm
                 synth.kv_dev(self.seed, synth.K_STREAM, kl, self.Bm, self.Hkv, 0, T, k, seq0=s0)
                 synth.kv_dev(self.seed, synth.V_STREAM, kl, self.Bm, self.Hkv, 0, T, v, seq0=s0)
-                synth.e_dev(self.seed, l, self.Bm, self.Hkv, 0, T, e, seq0=s0)
-                lay.append(k, v, e, T)
+                if self.head:
+                    lay.append_head(k, v, self.W[l][0], self.W[l][1], T)
+                else:
+                    synth.e_dev(self.seed, l, self.Bm, self.Hkv, 0, T, e, seq0=s0)
+                    lay.append(k, v, e, T)
         torch.cuda.synchronize()
         del k, v, e
 
@@ -135,7 +144,7 @@ class Workload:
         n, Um, L0 = self.n_steps, self.units_m, self.c["L"]
         self.q_bytes = self.Bm * self.Hq * D * 2
         self.kv_bytes = Um * D * 2
-        self.e_bytes = Um * 4
+        self.e_bytes = 0 if self.head else Um * 4
         self.part_in = self.q_bytes + 2 * self.kv_bytes + self.e_bytes
         self.step_in = self.L * self.micro * self.part_in
         self.inputs = torch.empty((n, self.step_in), dtype=torch.uint8, device=dev)
@@ -150,7 +159,8 @@ class Workload:
                 s0 = self.seq_base + m * self.Bm
                 synth.kv_dev(self.seed, synth.K_STREAM, kl, self.Bm, self.Hkv, L0, n, kk, seq0=s0)
                 synth.kv_dev(self.seed, synth.V_STREAM, kl, self.Bm, self.Hkv, L0, n, vv, seq0=s0)
-                synth.e_dev(self.seed, l, self.Bm, self.Hkv, L0, n, ee, seq0=s0)
+                if not self.head:
+                    synth.e_dev(self.seed, l, self.Bm, self.Hkv, L0, n, ee, seq0=s0)
                 base = (l * self.micro + m) * self.part_in
                 for t in range(n):
                     synth.q_dev(self.seed, l, self.Bm, self.Hq, t, qstate, qt, seq0=s0)
@@ -161,7 +171,8 @@ class Workload:
                     o += self.kv_bytes
                     row[o:o + self.kv_bytes].view(torch.int16).copy_(vv[:, t].reshape(-1))
                     o += self.kv_bytes
-                    row[o:o + self.e_bytes].view(torch.float32).copy_(ee[:, t])
+                    if self.e_bytes:
+                        row[o:o + self.e_bytes].view(torch.float32).copy_(ee[:, t])
         self.cur = torch.empty(self.step_in, dtype=torch.uint8, device=dev)
         self.out = torch.empty((self.L, self.B, self.Hq, D), dtype=torch.int16, device=dev)
         self.streams = [torch.cuda.Stream(device=dev) for _ in range(self.micro - 1)]
@@ -175,7 +186,7 @@ class Workload:
         o += self.kv_bytes
         v = buf[o:o + self.kv_bytes].view(torch.int16).view(self.units_m, 1, D)
         o += self.kv_bytes
-        e = buf[o:o + self.e_bytes].view(torch.float32).view(self.units_m, 1)
+        e = buf[o:o + self.e_bytes].view(torch.float32).view(self.units_m, 1) if self.e_bytes else None
         return q, k, v, e
 
     def out_view(self, l, m):
@@ -187,10 +198,14 @@ class Workload:
         lay = self.layers[l][m]
         q, k, v, e = self.views(buf, l, m)
         out = self.out_view(l, m)
+        if self.head:
+            w1, w2 = self.W[l]
+            append = ("append", lambda s: lay.append_head(k, v, w1, w2, 1, None, s))
+        else:
+            append = ("append", lambda s: lay.append(k, v, e, 1, None, s))
         if self.dense:  # the full-attention comparator: append, then attend to every token
-            return [("append", lambda s: lay.append(k, v, e, 1, None, s)),
-                    ("dense", lambda s: lay.dense_decode(q, out, s))]
-        calls = [("append", lambda s: lay.append(k, v, e, 1, None, s)), ("select", lambda s: lay.select(q, s))]
+            return [append, ("dense", lambda s: lay.dense_decode(q, out, s))]
+        calls = [append, ("select", lambda s: lay.select(q, s))]
         if self.c["offload"]:
             calls.append(("cache_sync", lambda s: lay.cache_sync(s)))
         calls.append(("decode", lambda s: lay.sparse_decode(q, out, s)))
@@ -435,14 +450,20 @@ def oracle_sample(c, groups, seed, n_units, n_steps, budget_s=25.0):
         kl = l % groups if c["offload"] else l
         K = synth.kv_rows(seed, synth.K_STREAM, kl, b, g, 0, L0 + n_steps)
         V = synth.kv_rows(seed, synth.V_STREAM, kl, b, g, 0, L0 + n_steps)
-        E = synth.e_rows(seed, l, b, g, 0, L0 + n_steps)
+        head = synth.head_weights(seed, l, c["Hkv"]) if c.get("head") else None
+        if head is not None:  # the prefill's logits come from the head too (untimed)
+            E = oracle.evict_head(V[:L0], head[0][g], head[1][g])
+        else:
+            E = synth.e_rows(seed, l, b, g, 0, L0 + n_steps)
         Q = np.stack([synth.q_steps(seed, l, b, g * G + h, n_steps)[1] for h in range(G)], axis=1)
         u = oracle.OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=cap, ck_bf16=c.get("ck_bf16", False),
                               fill=c.get("fill", False))
         u.prefill(K[:L0], V[:L0], E[:L0])
         for t in range(n_steps):
             t0 = time.perf_counter()
-            u.step(K[L0 + t], V[L0 + t], float(E[L0 + t]), Q[t])
+            e_t = (oracle.evict_head(V[L0 + t:L0 + t + 1], head[0][g], head[1][g])[0] if head is not None
+                   else E[L0 + t])
+            u.step(K[L0 + t], V[L0 + t], float(e_t), Q[t])
             total_t += time.perf_counter() - t0
             count += 1
             if total_t > budget_s:
@@ -651,7 +672,8 @@ def run_nosa(args, c, rank, world, dev):
         "config": {"workload": f"{args.workload}: " + describe(c, args.host_groups), "layers": c["layers"],
                    "batch": c["B"], "heads_q": c["Hq"], "heads_kv": c["Hkv"], "context": c["L"], "k_q": c["k_q"],
                    "k_e": c["k_e"], "offload": c["offload"], "pooled_keys": "bf16" if c.get("ck_bf16") else "fp32",
-                   "selection": "fill" if c.get("fill") else "union", "host_kv_groups": args.host_groups if c["offload"] else None,
+                   "selection": "fill" if c.get("fill") else "union",
+                   "eviction_logits": "fused head" if c.get("head") else "input", "host_kv_groups": args.host_groups if c["offload"] else None,
                    "cuda_graph": graph is not None, "micro_batches": wl.micro,
                    "l2": ("L2 flushed (256 MB write) before every timed step; steps timed one by one" if small else
                           f"inputs larger than L2: each step streams {step_bytes(wl) / 1e9:.2f} GB of pooled keys and KV blocks"),
@@ -767,6 +789,8 @@ def main():
     ap.add_argument("--ck-bf16", action="store_true", help="store pooled keys as bf16 instead of fp32")
     ap.add_argument("--kq-sweep", action="store_true",
                     help="gamma, misses and throughput against k_q/k, union and fill (one JSON line per point)")
+    ap.add_argument("--evict-head", action="store_true",
+                    help="compute the eviction logits with the fused synthetic eviction head inside append")
     ap.add_argument("--fill", action="store_true",
                     help="fill reading of the selection: Gamma_e fills the remainder outside Gamma_q")
     args = ap.parse_args()
@@ -775,6 +799,8 @@ def main():
         c["ck_bf16"] = True
     if args.fill:
         c["fill"] = True
+    if args.evict_head:
+        c["head"] = True
     if args.layers is not None:
         c["layers"] = args.layers
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -33,7 +33,7 @@ WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC = 0, 1, 2, 3
 
 # Every extern "C" symbol include/nosa.h declares.
 EXPORTS = ["nosa_validate_config", "nosa_state_bytes", "nosa_workspace_bytes", "nosa_state_init",
-           "nosa_compress_append", "nosa_select", "nosa_cache_sync", "nosa_sparse_decode",
+           "nosa_compress_append", "nosa_compress_append_head", "nosa_select", "nosa_cache_sync", "nosa_sparse_decode",
            "nosa_dense_decode", "nosa_read_error", "nosa_strerror", "nosa_select_noalloc"]
 NOALLOC_SELECT_SCRATCH = 1 << 20
 
@@ -85,6 +85,7 @@ def lib():
         L.nosa_workspace_bytes.restype = ctypes.c_size_t
         L.nosa_state_init.argtypes = [C, S, P]
         L.nosa_compress_append.argtypes = [C, S, P, P, P, ctypes.c_int32, P, P]
+        L.nosa_compress_append_head.argtypes = [C, S, P, P, P, P, ctypes.c_int32, P, P]
         L.nosa_select.argtypes = [C, S, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_cache_sync.argtypes = [C, S, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_sparse_decode.argtypes = [C, S, P, P, P, P, P, P, ctypes.c_size_t, P]
@@ -146,6 +147,12 @@ def nosa_state_init(cfg, st, stream=None):
 def nosa_compress_append(cfg, st, k_new, v_new, e_new, T, lens=None, stream=None):
     _check(lib().nosa_compress_append(ctypes.byref(cfg), ctypes.byref(st), _ptr(k_new), _ptr(v_new), _ptr(e_new),
                                       int(T), _ptr(lens), _stream(stream)), "nosa_compress_append")
+
+
+def nosa_compress_append_head(cfg, st, k_new, v_new, w1, w2, T, lens=None, stream=None):
+    _check(lib().nosa_compress_append_head(ctypes.byref(cfg), ctypes.byref(st), _ptr(k_new), _ptr(v_new), _ptr(w1),
+                                           _ptr(w2), int(T), _ptr(lens), _stream(stream)),
+           "nosa_compress_append_head")
 
 
 def nosa_select(cfg, st, q, sel, nsel, gq=None, ws=None, stream=None):
@@ -255,6 +262,10 @@ class NosaLayer:
     # one decode step = the four calls, in order
     def append(self, k_new, v_new, e_new, T=1, lens=None, stream=None):
         nosa_compress_append(self.cfg, self.state, k_new, v_new, e_new, T, lens, stream)
+
+    def append_head(self, k_new, v_new, w1, w2, T=1, lens=None, stream=None):
+        """Append with the eviction logits computed by the fused head (w1 fp32 [Hkv][D][128], w2 [Hkv][128])."""
+        nosa_compress_append_head(self.cfg, self.state, k_new, v_new, w1, w2, T, lens, stream)
 
     def select(self, q, stream=None):
         nosa_select(self.cfg, self.state, q, self.sel, self.nsel, self.gq, self.ws_select, stream)

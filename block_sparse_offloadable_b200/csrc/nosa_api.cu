@@ -262,9 +262,11 @@ int nosa_state_init(const nosa_config *c, const nosa_state *st, void *stream) {
     return ok ? NOSA_OK : NOSA_ERR_CUDA;
 }
 
-int nosa_compress_append(const nosa_config *c, const nosa_state *st, const uint16_t *k_new,
-                         const uint16_t *v_new, const float *e_new, int32_t T, const int32_t *lens,
-                         void *stream) {
+namespace {
+// nosa_compress_append with e_new given, or with the eviction head (w1, w2) computing it.
+int append_impl(const nosa_config *c, const nosa_state *st, const uint16_t *k_new, const uint16_t *v_new,
+                const float *e_new, const float *w1, const float *w2, int32_t T, const int32_t *lens,
+                void *stream) {
     Geo g;
     int rc;
     if ((rc = nosa_validate_config(c))) return rc;
@@ -272,8 +274,12 @@ int nosa_compress_append(const nosa_config *c, const nosa_state *st, const uint1
     if ((rc = check_state(c, st))) return rc;
     if (T < 1) return NOSA_ERR_ARG;
     if (T > c->max_ctx) return NOSA_ERR_CAPACITY;
-    if ((rc = check_dev(k_new, true)) || (rc = check_dev(v_new, true)) || (rc = check_dev(e_new, false)))
+    if ((rc = check_dev(k_new, true)) || (rc = check_dev(v_new, true))) return rc;
+    if (w1) {
+        if ((rc = check_dev(w1, true)) || (rc = check_dev(w2, true))) return rc;
+    } else if ((rc = check_dev(e_new, false))) {
         return rc;
+    }
     if (lens) {
         if (T == 1) return NOSA_ERR_ARG;
         if ((rc = check_dev(lens, false))) return rc;
@@ -282,7 +288,8 @@ int nosa_compress_append(const nosa_config *c, const nosa_state *st, const uint1
     if ((rc = store_addr(c, st, &s))) return rc;
     AppendParams p;
     memset(&p, 0, sizeof(p));
-    p.k_new = k_new; p.v_new = v_new; p.e_new = e_new; p.lens = lens;
+    p.k_new = k_new; p.v_new = v_new; p.e_new = w1 ? nullptr : e_new; p.lens = lens;
+    p.w1 = w1; p.w2 = w1 ? w2 : nullptr;
     p.store = s;
     p.cache = static_cast<uint8_t *>(c->offload ? st->cache : nullptr);
     p.e_store = st->evict_logit; p.ck = st->ck; p.blk_evict = st->blk_evict;
@@ -295,6 +302,21 @@ int nosa_compress_append(const nosa_config *c, const nosa_state *st, const uint1
     p.fill = (c->flags & NOSA_FLAG_FILL) != 0;
     p.pool = p.fill ? st->pool : nullptr; p.pool_n = p.fill ? st->pool_n : nullptr;
     return launch_append(p, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+int nosa_compress_append(const nosa_config *c, const nosa_state *st, const uint16_t *k_new,
+                         const uint16_t *v_new, const float *e_new, int32_t T, const int32_t *lens,
+                         void *stream) {
+    if (!e_new) return NOSA_ERR_ARG;
+    return append_impl(c, st, k_new, v_new, e_new, nullptr, nullptr, T, lens, stream);
+}
+
+int nosa_compress_append_head(const nosa_config *c, const nosa_state *st, const uint16_t *k_new,
+                              const uint16_t *v_new, const float *w1, const float *w2, int32_t T,
+                              const int32_t *lens, void *stream) {
+    if (!w1 || !w2) return NOSA_ERR_ARG;
+    return append_impl(c, st, k_new, v_new, nullptr, w1, w2, T, lens, stream);
 }
 
 int nosa_select(const nosa_config *c, const nosa_state *st, const uint16_t *q, int32_t *sel,

@@ -31,6 +31,13 @@ __device__ __forceinline__ void store_ck(const AppendParams &p, int64_t row, int
     }
 }
 
+// ---- eviction head: e_j = sum_h W2[h] softplus(v_j . W1[:, h]) -------------------------
+// fp64, every product and sum rounded on its own (no contraction), sums in index
+// order (d for the hidden pre-activations, h for the output), rounded once to fp32.
+__device__ __forceinline__ double softplus64(double x) {
+    return __dadd_rn(x > 0.0 ? x : 0.0, log1p(exp(-fabs(x))));
+}
+
 // Warp-cooperative argmin over Gamma_e by (E ascending, block id descending):
 // the member that leaves when a better block arrives.
 __device__ __forceinline__ void gamma_e_worst(const int32_t *ge, int32_t ne, const double *E,
@@ -52,10 +59,8 @@ __device__ __forceinline__ void gamma_e_worst(const int32_t *ge, int32_t ne, con
     }
 }
 
-__global__ void __launch_bounds__(128) append_decode_kernel(const AppendParams p) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int u = blockIdx.x * (blockDim.x >> 5) + warp;
-    if (u >= p.units) return;
+// One decode append of unit u by one warp, with the token's eviction logit e_tok.
+__device__ __forceinline__ void append_unit(const AppendParams &p, int32_t u, int lane, float e_tok) {
     const int32_t pos = p.seq_len[u];
     if (pos < 0 || pos >= p.max_ctx) {
         if (lane == 0) set_error(p.err, NOSA_EFLAG_CAPACITY);
@@ -103,7 +108,6 @@ __global__ void __launch_bounds__(128) append_decode_kernel(const AppendParams p
     const int64_t off = (lane < 16 ? 0 : kHalfBlockBytes) + (int64_t)w * kRowBytes + chunk * 16;
     *reinterpret_cast<uint4 *>(dst + off) = val;
     if (host) *reinterpret_cast<uint4 *>(host + off) = val;  // write-through over PCIe
-    const float e_tok = p.e_new[u];
     if (lane == 0) p.e_store[(int64_t)u * p.max_ctx + pos] = e_tok;
 
     // sub-block complete: its compressed key is the mean of its 16 keys (fp64 sum)
@@ -199,6 +203,69 @@ __global__ void __launch_bounds__(128) append_decode_kernel(const AppendParams p
     if (lane == 0) p.seq_len[u] = pos + 1;
 }
 
+__global__ void __launch_bounds__(128) append_decode_kernel(const AppendParams p) {
+    pdl_trigger();  // the select that follows waits for this grid anyway
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u = blockIdx.x * (blockDim.x >> 5) + warp;
+    if (u >= p.units) return;
+    append_unit(p, u, lane, p.e_new[u]);
+}
+
+// With the fused eviction head: one CTA of kHeadH threads per unit.  One bulk
+// copy stages W1 and W2 of the unit's kv head (64.5 KB) in shared memory;
+// thread h then runs hidden unit h's pre-activation in order over d, the 128
+// terms W2[h] softplus(z_h) are summed in order by one thread, and warp 0
+// appends the token with that logit.
+constexpr size_t kHeadDecSmem = (size_t)kD * kHeadH * 4 + kHeadH * 4 + kD * 8 + kHeadH * 8 + 16;
+
+__global__ void __launch_bounds__(kHeadH) append_head_decode_kernel(const AppendParams p) {
+    pdl_trigger();
+    pdl_wait();
+    extern __shared__ __align__(16) uint8_t smem[];
+    float *w1s = reinterpret_cast<float *>(smem);
+    float *w2s = w1s + kD * kHeadH;
+    double *vs = reinterpret_cast<double *>(w2s + kHeadH);
+    double *ts = vs + kD;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(ts + kHeadH);
+    __shared__ float s_e;
+    const int32_t u = blockIdx.x;
+    const int h = threadIdx.x, lane = threadIdx.x & 31;
+    const int32_t g = u % p.heads_kv;
+    if (h == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (h == 0) {
+        mbar_arrive_expect_tx(bar, (uint32_t)(kD * kHeadH * 4 + kHeadH * 4));
+        bulk_load(w1s, p.w1 + (int64_t)g * kD * kHeadH, kD * kHeadH * 4, bar);
+        bulk_load(w2s, p.w2 + (int64_t)g * kHeadH, kHeadH * 4, bar);
+    }
+    {  // the value row as fp64 (exact), while the weights are in flight
+        const uint16_t b = p.v_new[(int64_t)u * kD + h];
+        vs[h] = (double)__uint_as_float((uint32_t)b << 16);
+    }
+    const bool ok = mbar_wait(bar, 0);
+    if (__syncthreads_or(!ok)) {  // the whole CTA gives up together
+        if (!ok) mbar_wait(bar, 0);  // never leave with the copy in flight (bounded again)
+        if (h == 0) set_error(p.err, NOSA_EFLAG_TIMEOUT);
+        return;
+    }
+    double z = 0.0;
+#pragma unroll 8
+    for (int d = 0; d < kD; ++d) z = __dadd_rn(z, __dmul_rn(vs[d], (double)w1s[d * kHeadH + h]));
+    ts[h] = __dmul_rn((double)w2s[h], softplus64(z));
+    __syncthreads();
+    if (h == 0) {
+        double e = 0.0;
+        for (int i = 0; i < kHeadH; ++i) e = __dadd_rn(e, ts[i]);
+        s_e = __double2float_rn(e);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) append_unit(p, u, lane, s_e);
+}
+
 // ---- prefill ----------------------------------------------------------------------
 
 __device__ __forceinline__ int32_t unit_len(const AppendParams &p, int32_t u) {
@@ -225,7 +292,7 @@ __global__ void __launch_bounds__(256) prefill_store_kernel(const AppendParams p
         *reinterpret_cast<uint4 *>(p.store + ((int64_t)u * p.nblk + blk) * kBlockBytes + off) = val;
         if (p.offload && blk == (len - 1) >> 6)
             *reinterpret_cast<uint4 *>(p.cache + (int64_t)u * p.nslots * kBlockBytes + off) = val;
-        if (lane == 0) p.e_store[(int64_t)u * p.max_ctx + t] = p.e_new[(int64_t)u * p.T + t];
+        if (lane == 0 && !p.w1) p.e_store[(int64_t)u * p.max_ctx + t] = p.e_new[(int64_t)u * p.T + t];
     }
 }
 
@@ -256,7 +323,8 @@ __global__ void __launch_bounds__(256) prefill_pool_kernel(const AppendParams p)
         if ((blk + 1) * kBlock <= len) {
             double m = -__longlong_as_double(0x7FF0000000000000ll);
             if (lane < kSubPerBlock) {
-                const float *e = p.e_new + (int64_t)u * p.T + (int64_t)blk * kBlock + lane * kSub;
+                const float *e = (p.w1 ? p.e_store + (int64_t)u * p.max_ctx : p.e_new + (int64_t)u * p.T) +
+                                 (int64_t)blk * kBlock + lane * kSub;
                 double acc = 0.0;
                 for (int j = 0; j < kSub; ++j) acc += (double)e[j];
                 m = acc / kSub;
@@ -265,6 +333,79 @@ __global__ void __launch_bounds__(256) prefill_pool_kernel(const AppendParams p)
             m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             if (lane == 0) p.blk_evict[(int64_t)u * p.nblk + blk] = m;
         }
+    }
+}
+
+// Eviction head over the prefilled rows: a CTA stages W1 and W2 of its kv head in
+// shared memory and takes kHeadCtaRows rows of one unit; each warp runs 8 rows at
+// a time, a lane holding the pre-activations of hidden units lane + 32 i for all
+// 8 rows (32 fp64 accumulators); lane r then sums row r's 128 terms in order.
+constexpr int kHeadWarpRows = 8;
+constexpr int kHeadCtaRows = 256;
+constexpr int kHeadTStride = kHeadH + 2;  // doubles per row of t: rows land on distinct banks
+constexpr size_t kHeadSmem = (size_t)kD * kHeadH * 4 + kHeadH * 4 + 8 * kHeadWarpRows * kHeadTStride * 8;
+
+__global__ void __launch_bounds__(256) prefill_head_kernel(const AppendParams p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    float *w1s = reinterpret_cast<float *>(smem);
+    float *w2s = w1s + kD * kHeadH;
+    double *ts = reinterpret_cast<double *>(w2s + kHeadH);
+    const int32_t u = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (p.seq_len[u] != 0) return;  // prefill into a non-empty unit: flagged by prefill_gamma_kernel
+    const int32_t len = unit_len(p, u);
+    const int32_t r0 = blockIdx.x * kHeadCtaRows, r1 = min(r0 + kHeadCtaRows, len);
+    if (r0 >= r1) return;
+    const int32_t g = u % p.heads_kv;
+    const float4 *w1g = reinterpret_cast<const float4 *>(p.w1 + (int64_t)g * kD * kHeadH);
+    for (int i = threadIdx.x; i < kD * kHeadH / 4; i += blockDim.x) reinterpret_cast<float4 *>(w1s)[i] = w1g[i];
+    if (threadIdx.x < kHeadH) w2s[threadIdx.x] = p.w2[g * kHeadH + threadIdx.x];
+    __syncthreads();
+    double *tw = ts + warp * kHeadWarpRows * kHeadTStride;
+    for (int32_t rb = r0 + warp * kHeadWarpRows; rb < r1; rb += 8 * kHeadWarpRows) {
+        uint2 vv[kHeadWarpRows];
+#pragma unroll
+        for (int r = 0; r < kHeadWarpRows; ++r)
+            vv[r] = (rb + r < r1) ? reinterpret_cast<const uint2 *>(p.v_new + ((int64_t)u * p.T + rb + r) * kD)[lane]
+                                  : make_uint2(0u, 0u);
+        double z[kHeadWarpRows][4];
+#pragma unroll
+        for (int r = 0; r < kHeadWarpRows; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) z[r][i] = 0.0;
+        for (int d4 = 0; d4 < kD / 4; ++d4) {
+            uint32_t wx[kHeadWarpRows], wy[kHeadWarpRows];
+#pragma unroll
+            for (int r = 0; r < kHeadWarpRows; ++r) {
+                wx[r] = __shfl_sync(0xFFFFFFFFu, vv[r].x, d4);
+                wy[r] = __shfl_sync(0xFFFFFFFFu, vv[r].y, d4);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                double w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) w[i] = (double)w1s[(4 * d4 + k) * kHeadH + lane + 32 * i];
+#pragma unroll
+                for (int r = 0; r < kHeadWarpRows; ++r) {
+                    const uint32_t word = (k < 2) ? wx[r] : wy[r];
+                    const double v = (k & 1) ? bf16_hi(word) : bf16_lo(word);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) z[r][i] = __dadd_rn(z[r][i], __dmul_rn(v, w[i]));
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kHeadWarpRows; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                tw[r * kHeadTStride + 32 * i + lane] = __dmul_rn((double)w2s[32 * i + lane], softplus64(z[r][i]));
+        __syncwarp();
+        if (lane < kHeadWarpRows && rb + lane < r1) {
+            double e = 0.0;
+            for (int h = 0; h < kHeadH; ++h) e = __dadd_rn(e, tw[lane * kHeadTStride + h]);
+            p.e_store[(int64_t)u * p.max_ctx + rb + lane] = __double2float_rn(e);
+        }
+        __syncwarp();
     }
 }
 
@@ -327,15 +468,33 @@ __global__ void __launch_bounds__(256) prefill_gamma_kernel(const AppendParams p
 }
 
 int launch_append(const AppendParams &p, cudaStream_t stream) {
+    if (p.T == 1 && p.w1) {
+        if (cudaFuncSetAttribute(append_head_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kHeadDecSmem) != cudaSuccess)
+            return NOSA_ERR_CUDA;
+        return launch_pdl(append_head_decode_kernel, dim3(p.units), dim3(kHeadH), kHeadDecSmem, stream, p) ==
+                       cudaSuccess
+                   ? NOSA_OK
+                   : NOSA_ERR_CUDA;
+    }
     if (p.T == 1) {
         const int wpb = 4;
-        append_decode_kernel<<<(p.units + wpb - 1) / wpb, wpb * 32, 0, stream>>>(p);
-        return cudaGetLastError() == cudaSuccess ? NOSA_OK : NOSA_ERR_CUDA;
+        return launch_pdl(append_decode_kernel, dim3((p.units + wpb - 1) / wpb), dim3(wpb * 32), 0, stream, p) ==
+                       cudaSuccess
+                   ? NOSA_OK
+                   : NOSA_ERR_CUDA;
     }
     const int64_t rows = (int64_t)p.units * p.T;
     int64_t g = (rows + 7) / 8;
     if (g > 148 * 16) g = 148 * 16;
     prefill_store_kernel<<<(unsigned)g, 256, 0, stream>>>(p);
+    if (p.w1) {
+        if (cudaFuncSetAttribute(prefill_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kHeadSmem) != cudaSuccess)
+            return NOSA_ERR_CUDA;
+        dim3 hg((p.T + kHeadCtaRows - 1) / kHeadCtaRows, p.units);
+        prefill_head_kernel<<<hg, 256, kHeadSmem, stream>>>(p);
+    }
     const int64_t items = (int64_t)p.units * ((p.T + kBlock - 1) / kBlock);
     g = (items + 7) / 8;
     if (g > 148 * 16) g = 148 * 16;

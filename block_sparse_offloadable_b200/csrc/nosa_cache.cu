@@ -34,6 +34,8 @@ __device__ __forceinline__ uint32_t pack_miss(int32_t slot, int32_t blk) {
 }  // namespace
 
 __global__ void __launch_bounds__(kPlanWarps * 32) cache_plan_kernel(const CacheParams p) {
+    pdl_trigger();  // the gather's CTAs are small; they wait for this grid
+    pdl_wait();
     extern __shared__ uint32_t smem_words[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t u = blockIdx.x * kPlanWarps + warp;
@@ -107,6 +109,9 @@ __global__ void __launch_bounds__(kPlanWarps * 32) cache_plan_kernel(const Cache
 }
 
 __global__ void __launch_bounds__(kGatherThreads) cache_gather_kernel(const CacheParams p) {
+    // No early trigger: the decode that follows would hold most of each SM's
+    // shared memory for the whole (PCIe-bound) gather.
+    pdl_wait();
     extern __shared__ int32_t P[];  // [units + 1] prefix sums of the miss counts
     __shared__ int32_t s_wsum[kGatherThreads / 32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -182,10 +187,14 @@ int launch_cache_sync(const CacheParams &p, cudaStream_t stream) {
         cudaFuncSetAttribute(cache_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)plan_smem) != cudaSuccess)
         return NOSA_ERR_CUDA;
-    cache_plan_kernel<<<(p.units + kPlanWarps - 1) / kPlanWarps, kPlanWarps * 32, plan_smem, stream>>>(p);
+    if (launch_pdl(cache_plan_kernel, dim3((p.units + kPlanWarps - 1) / kPlanWarps), dim3(kPlanWarps * 32),
+                   plan_smem, stream, p) != cudaSuccess)
+        return NOSA_ERR_CUDA;
     const size_t gather_smem = ((size_t)p.units + 1) * sizeof(int32_t);
-    cache_gather_kernel<<<kNumSms * kGatherCtasPerSm, kGatherThreads, gather_smem, stream>>>(p);
-    return cudaGetLastError() == cudaSuccess ? NOSA_OK : NOSA_ERR_CUDA;
+    return launch_pdl(cache_gather_kernel, dim3(kNumSms * kGatherCtasPerSm), dim3(kGatherThreads), gather_smem,
+                      stream, p) == cudaSuccess
+               ? NOSA_OK
+               : NOSA_ERR_CUDA;
 }
 
 }  // namespace nosa

@@ -24,6 +24,7 @@ constexpr int kBlockBytes = 2 * kHalfBlockBytes;     // keys + values of a block
 constexpr int kMaxG = 8;                      // query heads per kv head handled by one tile
 constexpr int kMaxKq = 32;                    // Gamma_q fits one warp-wide sorted list
 constexpr int kMaxKe = 256;
+constexpr int kHeadH = NOSA_EVICT_HIDDEN;             // hidden width of the eviction head
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at 2 GHz: bound on every mbarrier wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -222,6 +223,19 @@ __device__ __forceinline__ void list_merge(uint64_t &list, uint64_t other, int l
     }
     list = m;
 }
+
+// ---- programmatic dependent launch ---------------------------------------------
+// Every kernel of the decode chain is launched with programmatic stream
+// serialization and waits here before its first global access: the wait returns
+// once the previous kernel on the stream has completed and its writes are
+// visible, so ordering is unchanged while the launch and CTA setup overlap the
+// previous kernel's tail.  Every CTA waits, so completion stays transitive.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel on the stream launch now (its CTAs then wait in pdl_wait).
+// Used by kernels whose successor is small or short-waiting, never before a
+// long-running kernel's successor could hold SM resources needed elsewhere.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bits) {
     if (err) atomicOr(err, bits);

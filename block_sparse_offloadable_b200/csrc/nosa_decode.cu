@@ -206,6 +206,8 @@ int decode_ctas() { return kNumSms; }
 
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p) {
+    pdl_trigger();  // the next append's CTAs are tiny; they wait for this grid
+    pdl_wait();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *tiles = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -519,8 +521,10 @@ int launch_decode(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t s
     if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return NOSA_ERR_CUDA;
-    decode_kernel<<<decode_ctas(), kDecThreads, smem, stream>>>(tmap, p);
-    return cudaGetLastError() == cudaSuccess ? NOSA_OK : NOSA_ERR_CUDA;
+    return launch_pdl(decode_kernel, dim3(decode_ctas()), dim3(kDecThreads), smem, stream, tmap, p) ==
+                   cudaSuccess
+               ? NOSA_OK
+               : NOSA_ERR_CUDA;
 }
 
 }  // namespace nosa

@@ -2,6 +2,8 @@
 // libnosa translation units (not part of the C ABI).
 #pragma once
 
+#include <utility>
+
 #include "nosa_common.cuh"
 
 namespace nosa {
@@ -9,7 +11,9 @@ namespace nosa {
 struct AppendParams {
     const uint16_t *k_new;   // [u][T][D]
     const uint16_t *v_new;   // [u][T][D]
-    const float *e_new;      // [u][T]
+    const float *e_new;      // [u][T], or null when the eviction head computes e
+    const float *w1;         // eviction head: [Hkv][D][kHeadH] or null
+    const float *w2;         // [Hkv][kHeadH]
     const int32_t *lens;     // [B] or null (prefill)
     uint8_t *store;          // device address of the KV store (device memory or mapped host)
     uint8_t *cache;          // offload cache or null
@@ -106,6 +110,24 @@ inline int best_chunks(int64_t units, int64_t work, int64_t slots, int64_t ovh, 
         if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_n = n; }
     }
     return (int)best_n;
+}
+
+// Launch with programmatic stream serialization (the kernel must call pdl_wait()
+// before touching global memory).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace nosa

@@ -134,6 +134,8 @@ template <typename T>
 __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectParams p) {
     constexpr int kSelS = SelGeo<T>::kStages;
     constexpr int kStageBytes = stage_bytes<T>();
+    pdl_trigger();  // the successor (cache plan or decode) waits for this grid anyway
+    pdl_wait();
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *tiles = smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(tiles + kSelS * kStageBytes);
@@ -330,8 +332,9 @@ int launch_select_t(const SelectParams &p, cudaStream_t stream) {
                              (int)smem) != cudaSuccess)
         return NOSA_ERR_CUDA;
     dim3 grid(p.nchunks, p.units);
-    select_kernel<T><<<grid, (kSelW + 1) * 32, smem, stream>>>(p);
-    return cudaGetLastError() == cudaSuccess ? NOSA_OK : NOSA_ERR_CUDA;
+    return launch_pdl(select_kernel<T>, grid, dim3((kSelW + 1) * 32), smem, stream, p) == cudaSuccess
+               ? NOSA_OK
+               : NOSA_ERR_CUDA;
 }
 
 int launch_select(const SelectParams &p, cudaStream_t stream) {

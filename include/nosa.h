@@ -210,6 +210,30 @@ int nosa_compress_append(const nosa_config *cfg, const nosa_state *st, const uin
                          const uint16_t *v_new, const float *e_new, int32_t T, const int32_t *lens,
                          void *stream);
 
+/* Hidden width of the eviction head of nosa_compress_append_head. */
+#define NOSA_EVICT_HIDDEN 128
+
+/*
+ * a1 with the eviction head fused in.  NOSA pages: montaan.com summary of
+ * 2510.13602, "Key Design Components" item 3 (Equation 4: the eviction score
+ * of token j is tau(v_j W1) W2 with tau = softplus) and "System Optimization
+ * (NOSI)" item 1 (the eviction head fused into the kernel that splits QKV).
+ *
+ *   w1  device fp32 [Hkv][D][NOSA_EVICT_HIDDEN]   one head per kv head (row d, column h),
+ *       16-byte aligned
+ *   w2  device fp32 [Hkv][NOSA_EVICT_HIDDEN], 16-byte aligned
+ *
+ * As nosa_compress_append, but the eviction logit of every appended token is
+ * computed from its value row in the same launch instead of being passed in:
+ *   e_j = sum_h w2[g][h] * softplus( sum_d v_j[d] * w1[g][d][h] ),
+ * in fp64 with each product and sum rounded on its own, sums in index order,
+ * softplus(x) = max(x, 0) + log1p(exp(-|x|)), rounded once to fp32 and stored
+ * in evict_logit.  Same device errors as nosa_compress_append.
+ */
+int nosa_compress_append_head(const nosa_config *cfg, const nosa_state *st, const uint16_t *k_new,
+                              const uint16_t *v_new, const float *w1, const float *w2, int32_t T,
+                              const int32_t *lens, void *stream);
+
 /*
  * a2 + a3 -- two-stage block scoring and dual selection.  NOSA pages:
  * wmrh.cn NOSA-1B release ("two-stage attention: select Top-K blocks with

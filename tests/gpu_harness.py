@@ -18,6 +18,7 @@ import numpy as np
 import torch
 
 import block_sparse_offloadable_b200 as nosa
+import oracle
 import synth
 from oracle import OracleUnit
 
@@ -27,7 +28,7 @@ MAX_ABS, MEAN_ABS, REL_L2 = 1e-2, 1e-3, 1e-2
 
 class Scenario:
     def __init__(self, B, Hq, Hkv, k_q, k_e, L0, steps, offload=False, seed=0, layer=0, lens=None,
-                 max_ctx=None, dense=False, ck_bf16=False, fill=False):
+                 max_ctx=None, dense=False, ck_bf16=False, fill=False, head=False):
         self.B, self.Hq, self.Hkv, self.k_q, self.k_e = B, Hq, Hkv, k_q, k_e
         self.G = Hq // Hkv
         self.units = B * Hkv
@@ -38,6 +39,8 @@ class Scenario:
         self.dense = dense
         self.ck_bf16 = ck_bf16
         self.fill = fill
+        self.head = head  # eviction logits from the fused head (synthetic weights) instead of inputs
+        self.W = synth.head_weights(seed, layer, Hkv) if head else None
 
     def cfg(self):
         return nosa.make_config(self.B, self.Hq, self.Hkv, self.k_q, self.k_e, self.max_ctx, self.offload,
@@ -45,7 +48,8 @@ class Scenario:
 
 
 def unit_data(sc):
-    """Host K, V [units][Lmax][D] (bf16 bits), e [units][Lmax] and queries [steps][B][Hq][D]."""
+    """Host K, V [units][Lmax][D] (bf16 bits), e [units][Lmax] and queries [steps][B][Hq][D].
+    With the eviction head, e is the oracle's head output on V (the GPU computes its own)."""
     D = 128
     K = np.empty((sc.units, sc.Lmax, D), np.uint16)
     V = np.empty_like(K)
@@ -54,7 +58,10 @@ def unit_data(sc):
         b, g = divmod(u, sc.Hkv)
         K[u] = synth.kv_rows(sc.seed, synth.K_STREAM, sc.layer, b, g, 0, sc.Lmax)
         V[u] = synth.kv_rows(sc.seed, synth.V_STREAM, sc.layer, b, g, 0, sc.Lmax)
-        E[u] = synth.e_rows(sc.seed, sc.layer, b, g, 0, sc.Lmax)
+        if sc.head:
+            E[u] = oracle.evict_head(V[u], sc.W[0][g], sc.W[1][g])
+        else:
+            E[u] = synth.e_rows(sc.seed, sc.layer, b, g, 0, sc.Lmax)
     Q = np.empty((sc.steps, sc.B, sc.Hq, D), np.uint16)
     for b in range(sc.B):
         for h in range(sc.Hq):
@@ -70,6 +77,16 @@ def run_gpu(sc, data):
     """Drive the four entry points for every step; return per-step host copies."""
     K, V, E, Q = data
     lay = nosa.NosaLayer(sc.cfg())
+    if sc.head:
+        w1 = torch.from_numpy(sc.W[0]).cuda()
+        w2 = torch.from_numpy(sc.W[1]).cuda()
+
+    def append(k, v, e, T, lens=None):
+        if sc.head:
+            lay.append_head(k, v, w1, w2, T, lens)
+        else:
+            lay.append(k, v, e, T, lens)
+
     T = max(sc.lens)
     lens = np.array(sc.lens, np.int32)
     if T > 0:
@@ -80,8 +97,8 @@ def run_gpu(sc, data):
             n = lens[u // sc.Hkv]
             kp[u, :n], vp[u, :n], ep[u, :n] = K[u, :n], V[u, :n], E[u, :n]
         ragged = len(set(sc.lens)) > 1
-        lay.append(_dev16(kp), _dev16(vp), torch.from_numpy(ep).cuda(), T,
-                   torch.from_numpy(lens).cuda() if ragged else None)
+        append(_dev16(kp), _dev16(vp), torch.from_numpy(ep).cuda(), T,
+               torch.from_numpy(lens).cuda() if ragged else None)
     res = {k: [] for k in ("sel", "nsel", "gq", "ge", "gn", "out", "nf", "dense")}
     for t in range(sc.steps):
         idx = lens.repeat(sc.Hkv) + t  # position of this step's token, per unit
@@ -90,7 +107,7 @@ def run_gpu(sc, data):
         en = torch.from_numpy(np.ascontiguousarray(E[np.arange(sc.units), idx][:, None])).cuda()
         q = _dev16(Q[t])
         out = torch.empty((sc.B, sc.Hq, 128), dtype=torch.int16, device="cuda")
-        lay.append(kn, vn, en, 1)
+        append(kn, vn, en, 1)
         lay.select(q)
         if sc.offload:
             lay.cache_sync()
@@ -110,6 +127,7 @@ def run_gpu(sc, data):
     res["err"] = lay.read_error()
     res["seq_len"] = lay.seq_len.cpu().numpy()
     res["ck"] = lay.ck.cpu().numpy()
+    res["e"] = lay.evict_logit.view(sc.units, -1).cpu().numpy()
     return res
 
 

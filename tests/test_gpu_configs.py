@@ -15,6 +15,7 @@ import pytest
 import torch
 
 import bench
+import oracle
 import synth
 from oracle import OracleUnit
 from tests import gpu_harness as H
@@ -70,7 +71,11 @@ def run_config(c, steps, seqs=None, seed=0, micro=1, dense_step=None, name=None)
     for (b, g) in units:
         K = synth.kv_rows(seed, synth.K_STREAM, wl.kv_layer(0), b, g, 0, L0 + steps)
         V = synth.kv_rows(seed, synth.V_STREAM, wl.kv_layer(0), b, g, 0, L0 + steps)
-        E = synth.e_rows(seed, 0, b, g, 0, L0 + steps)
+        if c.get("head"):
+            W1, W2 = synth.head_weights(seed, 0, c["Hkv"])
+            E = oracle.evict_head(V, W1[g], W2[g])
+        else:
+            E = synth.e_rows(seed, 0, b, g, 0, L0 + steps)
         Q = np.stack([synth.q_steps(seed, 0, b, g * G + h, steps)[1] for h in range(G)], axis=1)
         o = OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=wl.max_ctx, ck_bf16=c.get("ck_bf16", False),
                        fill=c.get("fill", False))
