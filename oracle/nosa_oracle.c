@@ -44,7 +44,8 @@
  *     it is always kept and not counted in k.
  *   - Ties in any top-k go to the lower block index.
  *   - After a prefill, Gamma_e is the plain top-k_e; nothing is marked
- *     dropped before the first decode step.
+ *     dropped before the first decode step; the block cache holds Gamma_e and
+ *     the local block (the prefill has them at hand, so no transfer).
  *   - Decode order: append the token, then select, then attend (the new token
  *     attends to itself).
  *
@@ -250,10 +251,12 @@ int nosa_oracle_prefill(nosa_oracle_unit *u, const uint16_t *K, const uint16_t *
     memset(u->ge_inc, 0, (size_t)(u->cap / u->block));
     for (int32_t i = 0; i < n; ++i) u->ge_inc[ids[i]] = 1;
     u->n_ge_inc = n;
-    free(ids);
-    /* the block cache starts holding only the local block (written during prefill) */
+    /* the block cache starts holding Gamma_e and the local block: the prefill has
+       every block at hand, so these cost no transfer */
     memset(u->resident, 0, (size_t)(u->cap / u->block));
+    for (int32_t i = 0; i < n; ++i) u->resident[ids[i]] = 1;
     if (u->L > 0) u->resident[(u->L - 1) / u->block] = 1;
+    free(ids);
     u->have_prev = 0;
     return 0;
 }

@@ -152,7 +152,7 @@ def test_locality_bound_is_tight_with_alternating_queries():
         assert r["ge"].tolist() == [0, 1, 2, 3, 4, 5]
         assert r["gq"].tolist() == ([10, 11] if t % 2 == 0 else [20, 21])
         if t == 0:
-            assert r["n_fetch"] == 8  # cold cache: only the local block is resident after prefill
+            assert r["n_fetch"] == 2  # the prefill leaves Gamma_e and the local block resident
         else:
             assert r["n_overlap"] == 6 and r["gamma"] == 0.75 and r["n_fetch"] == 2
     assert u.violations()["gamma"] == 0
