@@ -63,6 +63,8 @@ def describe(c, groups):
         s += ", fill reading of the selection"
     if c.get("head"):
         s += ", eviction logits from the fused synthetic eviction head"
+    if c.get("split"):
+        s += ", decode split: Gamma_e + local attended while select and the cache sync run"
     return s
 
 
@@ -111,6 +113,7 @@ class Workload:
                         for m in range(micro)] for l in range(self.L)]
         # the fused eviction head: synthetic weights per layer (e is then computed, not an input)
         self.head = bool(c.get("head", False))
+        self.split = bool(c.get("split", False))  # decode Gamma_e + local while select / cache sync run
         self.W = [tuple(torch.from_numpy(w).to(dev) for w in synth.head_weights(seed, l, self.Hkv))
                   for l in range(self.L)] if self.head else None
         self._prefill(dev)
@@ -176,6 +179,7 @@ class Workload:
         self.cur = torch.empty(self.step_in, dtype=torch.uint8, device=dev)
         self.out = torch.empty((self.L, self.B, self.Hq, D), dtype=torch.int16, device=dev)
         self.streams = [torch.cuda.Stream(device=dev) for _ in range(self.micro - 1)]
+        self.side = [torch.cuda.Stream(device=dev) for _ in range(self.micro)] if self.split else []
         torch.cuda.synchronize()
 
     def views(self, buf, l, m=0):
@@ -193,7 +197,9 @@ class Workload:
         return self.out[l, m * self.Bm:(m + 1) * self.Bm]
 
     def kernel_calls(self, l, m, buf=None):
-        """(name, call) of one layer's step for micro-batch m, in order."""
+        """(name, call) of one layer's step for micro-batch m, in order.  With the split decode,
+        ("fork", None) starts the side stream, calls named "resident" run on it, and ("join", None)
+        joins it back before the rest of the decode."""
         buf = self.cur if buf is None else buf
         lay = self.layers[l][m]
         q, k, v, e = self.views(buf, l, m)
@@ -205,10 +211,16 @@ class Workload:
             append = ("append", lambda s: lay.append(k, v, e, 1, None, s))
         if self.dense:  # the full-attention comparator: append, then attend to every token
             return [append, ("dense", lambda s: lay.dense_decode(q, out, s))]
-        calls = [append, ("select", lambda s: lay.select(q, s))]
+        calls = [append]
+        if self.split:
+            calls += [("fork", None), ("resident", lambda s: lay.decode_resident(q, s))]
+        calls.append(("select", lambda s: lay.select(q, s)))
         if self.c["offload"]:
             calls.append(("cache_sync", lambda s: lay.cache_sync(s)))
-        calls.append(("decode", lambda s: lay.sparse_decode(q, out, s)))
+        if self.split:
+            calls += [("join", None), ("rest", lambda s: lay.decode_rest(q, out, s))]
+        else:
+            calls.append(("decode", lambda s: lay.sparse_decode(q, out, s)))
         return calls
 
     def launch_step(self, buf=None, events=None):
@@ -222,6 +234,8 @@ class Workload:
             for l in range(self.L):
                 for m in range(self.micro):
                     for name, fn in self.kernel_calls(l, m, buf):
+                        if fn is None:
+                            continue
                         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                         e0.record()
                         fn(cur)
@@ -233,8 +247,13 @@ class Workload:
             s.wait_stream(cur)
         for l in range(self.L):
             for m in range(self.micro):
-                for _, fn in self.kernel_calls(l, m, buf):
-                    fn(streams[m])
+                for name, fn in self.kernel_calls(l, m, buf):
+                    if name == "fork":
+                        self.side[m].wait_stream(streams[m])
+                    elif name == "join":
+                        streams[m].wait_stream(self.side[m])
+                    else:
+                        fn(self.side[m] if name == "resident" else streams[m])
         for s in self.streams:
             cur.wait_stream(s)
 
@@ -271,8 +290,8 @@ class Workload:
 
     @property
     def launches_per_step(self):
-        # append, select, [cache plan, cache gather], decode
-        return self.L * self.micro * (5 if self.c["offload"] else 3)
+        # append, select, [cache plan, cache gather], decode (split: resident + rest)
+        return self.L * self.micro * ((5 if self.c["offload"] else 3) + (1 if self.split else 0))
 
 
 # ---------------------------------------------------------------------------------------
@@ -308,8 +327,8 @@ def step_bytes(wl):
 
 
 def time_idempotent(wl, name, reps, flush=None):
-    """Average device time of one launch of an idempotent kernel (select or decode):
-    a CUDA graph of that kernel for every layer, replayed back to back."""
+    """Average device time of one launch of an idempotent kernel (select, decode, or the split
+    decode's resident / rest passes): a CUDA graph of that kernel for every layer, replayed back to back."""
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -320,6 +339,10 @@ def time_idempotent(wl, name, reps, flush=None):
                 q, _, _, _ = wl.views(wl.cur, l, m)
                 if name == "select":
                     lay.select(q)
+                elif name == "resident":
+                    lay.decode_resident(q)
+                elif name == "rest":
+                    lay.decode_rest(q, wl.out_view(l, m))
                 else:
                     lay.sparse_decode(q, wl.out_view(l, m))
     torch.cuda.synchronize()
@@ -588,9 +611,10 @@ def run_nosa(args, c, rank, world, dev):
     for name, l, a, b in events:
         kt.setdefault(name, []).append(a.elapsed_time(b))
     # select and decode are idempotent: replace their event times by graph-replay times
-    for name in ("select", "decode"):
-        per = time_idempotent(wl, name, reps=3, flush=flush)
-        kt[name] = [per] * len(kt[name])
+    for name in ("select", "decode", "resident", "rest"):
+        if name in kt:
+            per = time_idempotent(wl, name, reps=3, flush=flush)
+            kt[name] = [per] * len(kt[name])
     nsel_mean = nsel_sum / max(nsel_n, 1)
     hbm_peak, peak_kind = load_peaks()
     U, Lctx = wl.units_m, c["L"] + step_i
@@ -600,6 +624,9 @@ def run_nosa(args, c, rank, world, dev):
         "decode": U * nsel_mean * (64 * D * 2 * 2 + 64 * 4) + 2 * wl.Bm * c["Hq"] * D * 2,
         "append": U * (2 * D * 2 + 4),
     }
+    n_res = min(c["k_e"], nb_c) + 1  # Gamma_e + the local block
+    algo["resident"] = U * n_res * (64 * D * 2 * 2 + 64 * 4) + wl.Bm * c["Hq"] * D * 2
+    algo["rest"] = U * max(nsel_mean - n_res, 0) * (64 * D * 2 * 2 + 64 * 4) + 2 * wl.Bm * c["Hq"] * D * 2
     kern = {}
     for name, ts in kt.items():
         avg = sum(ts) / len(ts)
@@ -673,7 +700,8 @@ def run_nosa(args, c, rank, world, dev):
                    "batch": c["B"], "heads_q": c["Hq"], "heads_kv": c["Hkv"], "context": c["L"], "k_q": c["k_q"],
                    "k_e": c["k_e"], "offload": c["offload"], "pooled_keys": "bf16" if c.get("ck_bf16") else "fp32",
                    "selection": "fill" if c.get("fill") else "union",
-                   "eviction_logits": "fused head" if c.get("head") else "input", "host_kv_groups": args.host_groups if c["offload"] else None,
+                   "eviction_logits": "fused head" if c.get("head") else "input",
+                   "decode": "split (resident during select / cache sync, then rest)" if c.get("split") else "one pass", "host_kv_groups": args.host_groups if c["offload"] else None,
                    "cuda_graph": graph is not None, "micro_batches": wl.micro,
                    "l2": ("L2 flushed (256 MB write) before every timed step; steps timed one by one" if small else
                           f"inputs larger than L2: each step streams {step_bytes(wl) / 1e9:.2f} GB of pooled keys and KV blocks"),
@@ -791,6 +819,8 @@ def main():
                     help="gamma, misses and throughput against k_q/k, union and fill (one JSON line per point)")
     ap.add_argument("--evict-head", action="store_true",
                     help="compute the eviction logits with the fused synthetic eviction head inside append")
+    ap.add_argument("--split", action="store_true",
+                    help="split decode: attend Gamma_e + the local block while select and the cache sync run")
     ap.add_argument("--fill", action="store_true",
                     help="fill reading of the selection: Gamma_e fills the remainder outside Gamma_q")
     args = ap.parse_args()
@@ -801,6 +831,8 @@ def main():
         c["fill"] = True
     if args.evict_head:
         c["head"] = True
+    if args.split:
+        c["split"] = True
     if args.layers is not None:
         c["layers"] = args.layers
     world = int(os.environ.get("WORLD_SIZE", "1"))

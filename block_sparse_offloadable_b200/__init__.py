@@ -29,12 +29,13 @@ EFLAG_CAPACITY, EFLAG_TIMEOUT, EFLAG_NOSLOT, EFLAG_STATE = 1, 2, 4, 8
 FLAG_CK_BF16, FLAG_FILL = 1, 2
 (BUF_KV_STORE, BUF_EVICT_LOGIT, BUF_CK, BUF_BLK_EVICT, BUF_GAMMA_E, BUF_GAMMA_N, BUF_SEQ_LEN, BUF_CACHE,
  BUF_SLOT_BLOCK, BUF_BLOCK_SLOT, BUF_ERR, BUF_POOL, BUF_POOL_N) = range(13)
-WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC = 0, 1, 2, 3
+WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC, WS_SPLIT = 0, 1, 2, 3, 4
 
 # Every extern "C" symbol include/nosa.h declares.
 EXPORTS = ["nosa_validate_config", "nosa_state_bytes", "nosa_workspace_bytes", "nosa_state_init",
            "nosa_compress_append", "nosa_compress_append_head", "nosa_select", "nosa_cache_sync", "nosa_sparse_decode",
-           "nosa_dense_decode", "nosa_read_error", "nosa_strerror", "nosa_select_noalloc"]
+           "nosa_dense_decode", "nosa_decode_resident", "nosa_decode_rest", "nosa_read_error", "nosa_strerror",
+           "nosa_select_noalloc"]
 NOALLOC_SELECT_SCRATCH = 1 << 20
 
 
@@ -89,6 +90,8 @@ def lib():
         L.nosa_select.argtypes = [C, S, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_cache_sync.argtypes = [C, S, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_sparse_decode.argtypes = [C, S, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.nosa_decode_resident.argtypes = [C, S, P, P, ctypes.c_size_t, P, ctypes.c_size_t, P]
+        L.nosa_decode_rest.argtypes = [C, S, P, P, P, ctypes.c_size_t, P, P, ctypes.c_size_t, P]
         L.nosa_dense_decode.argtypes = [C, S, P, P, P, ctypes.c_size_t, P]
         L.nosa_read_error.argtypes = [S, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P]
         L.nosa_select_noalloc.argtypes = [C, S, P, P, P, P, P]
@@ -180,6 +183,21 @@ def nosa_sparse_decode(cfg, st, q, sel, nsel, block_table, out, ws=None, stream=
            "nosa_sparse_decode")
 
 
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def nosa_decode_resident(cfg, st, q, split, ws=None, stream=None):
+    _check(lib().nosa_decode_resident(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(split), _nbytes(split),
+                                      _ptr(ws), _nbytes(ws), _stream(stream)), "nosa_decode_resident")
+
+
+def nosa_decode_rest(cfg, st, q, gq, split, out, ws=None, stream=None):
+    _check(lib().nosa_decode_rest(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(gq), _ptr(split),
+                                  _nbytes(split), _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "nosa_decode_rest")
+
+
 def nosa_dense_decode(cfg, st, q, out, ws=None, stream=None):
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib().nosa_dense_decode(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(out), _ptr(ws), nbytes,
@@ -257,6 +275,7 @@ class NosaLayer:
         self.ws_decode = ws(WS_SPARSE_DECODE)
         self.ws_dense = None if cfg.offload else ws(WS_DENSE_DECODE)
         self.ws_cache = ws(WS_CACHE_SYNC)
+        self.split = None if cfg.flags & FLAG_FILL else ws(WS_SPLIT)
         nosa_state_init(cfg, self.state)
 
     # one decode step = the four calls, in order
@@ -277,6 +296,14 @@ class NosaLayer:
     def sparse_decode(self, q, out, stream=None):
         bt = self.block_table if self.cfg.offload else None
         nosa_sparse_decode(self.cfg, self.state, q, self.sel, self.nsel, bt, out, self.ws_decode, stream)
+
+    def decode_resident(self, q, stream=None):
+        """Attention over Gamma_e + the local block, right after append (may overlap select / cache_sync)."""
+        nosa_decode_resident(self.cfg, self.state, q, self.split, self.ws_decode, stream)
+
+    def decode_rest(self, q, out, stream=None):
+        """Attention over the rest of Gamma_q, merged with decode_resident's state, into out."""
+        nosa_decode_rest(self.cfg, self.state, q, self.gq, self.split, out, self.ws_decode, stream)
 
     def dense_decode(self, q, out, stream=None):
         nosa_dense_decode(self.cfg, self.state, q, out, self.ws_dense, stream)

@@ -122,6 +122,9 @@ int select_nchunks(const nosa_config *c, const Geo &g) {
     return n < 1 ? 1 : (int)n;
 }
 
+// Words of the per-unit block bitmap in the split-decode buffer.
+size_t split_bits_words(const Geo &g) { return (size_t)g.nblk / 32 + 1; }
+
 size_t ws_bytes_of(const nosa_config *c, int which) {
     Geo g;
     if (!geo_of(c, &g)) return 0;
@@ -134,6 +137,9 @@ size_t ws_bytes_of(const nosa_config *c, int which) {
         return counters + (size_t)decode_ctas() * 2 * kPartFloats * sizeof(float);
     if (which == NOSA_WS_CACHE_SYNC)
         return c->offload ? counters + (size_t)g.units * g.max_sel * sizeof(uint32_t) : 0;
+    if (which == NOSA_WS_SPLIT)
+        return align256((size_t)g.units * kPartFloats * sizeof(float)) +
+               (size_t)g.units * split_bits_words(g) * sizeof(uint32_t);
     return 0;
 }
 
@@ -144,20 +150,28 @@ int check_ws(const nosa_config *c, int which, void *ws, size_t ws_bytes) {
     return check_dev(ws, true);
 }
 
-int run_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q, const int32_t *sel,
-               const int32_t *nsel, const int32_t *block_table, uint16_t *out, void *ws,
-               size_t ws_bytes, void *stream, bool dense) {
+// One decode launch in the given mode (kMode*): the work list, where the blocks
+// live, and where the result goes differ; see nosa_decode.cu.
+int run_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q, int mode, const int32_t *sel,
+               const int32_t *nsel, const int32_t *block_table, const int32_t *gq, void *split,
+               size_t split_bytes, uint16_t *out, void *ws, size_t ws_bytes, void *stream) {
     Geo g;
     int rc;
     if ((rc = nosa_validate_config(c))) return rc;
     geo_of(c, &g);
     if ((rc = check_state(c, st))) return rc;
-    if ((rc = check_dev(q, true)) || (rc = check_dev(out, true))) return rc;
-    if (!dense) {
+    if ((rc = check_dev(q, true))) return rc;
+    if (mode != kModeResident && (rc = check_dev(out, true))) return rc;
+    if (mode == kModeSel) {
         if ((rc = check_dev(sel, false)) || (rc = check_dev(nsel, false))) return rc;
         if (c->offload && (rc = check_dev(block_table, false))) return rc;
     }
-    const int which = dense ? NOSA_WS_DENSE_DECODE : NOSA_WS_SPARSE_DECODE;
+    if (mode == kModeResident || mode == kModeRest) {
+        if (c->flags & NOSA_FLAG_FILL) return NOSA_ERR_UNSUPPORTED;  // Gamma_e needs Gamma_q there
+        if ((rc = check_ws(c, NOSA_WS_SPLIT, split, split_bytes))) return rc;
+        if (mode == kModeRest && c->k_q > 0 && (rc = check_dev(gq, false))) return rc;
+    }
+    const int which = mode == kModeDense ? NOSA_WS_DENSE_DECODE : NOSA_WS_SPARSE_DECODE;
     if ((rc = check_ws(c, which, ws, ws_bytes))) return rc;
 
     const void *base;
@@ -177,9 +191,20 @@ int run_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q, co
     DecodeParams p;
     memset(&p, 0, sizeof(p));
     p.q = q;
-    p.sel = dense ? nullptr : sel;
-    p.nsel = dense ? nullptr : nsel;
-    p.block_table = (dense || !c->offload) ? nullptr : block_table;
+    p.mode = mode;
+    p.sel = mode == kModeSel ? sel : nullptr;
+    p.nsel = mode == kModeSel ? nsel : nullptr;
+    p.block_table = (mode == kModeSel && c->offload) ? block_table : nullptr;
+    if (mode == kModeResident || mode == kModeRest) {
+        p.gamma_e = st->gamma_e; p.gamma_n = st->gamma_n; p.k_e = c->k_e;
+        p.gq = c->k_q > 0 ? gq : nullptr; p.k_q = c->k_q;
+        p.block_slot = c->offload ? st->block_slot : nullptr;
+        p.nblk = (int32_t)g.nblk;
+        p.bits_words = (int32_t)split_bits_words(g);
+        p.res_part = static_cast<float *>(split);
+        p.res_bits = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(split) +
+                                                  align256((size_t)g.units * kPartFloats * sizeof(float)));
+    }
     p.e = st->evict_logit;
     p.seq_len = st->seq_len;
     p.out = out;
@@ -382,13 +407,27 @@ int nosa_cache_sync(const nosa_config *c, const nosa_state *st, const int32_t *s
 int nosa_sparse_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q,
                        const int32_t *sel, const int32_t *nsel, const int32_t *block_table,
                        uint16_t *out, void *ws, size_t ws_bytes, void *stream) {
-    return run_decode(c, st, q, sel, nsel, block_table, out, ws, ws_bytes, stream, false);
+    return run_decode(c, st, q, kModeSel, sel, nsel, block_table, nullptr, nullptr, 0, out, ws, ws_bytes, stream);
+}
+
+int nosa_decode_resident(const nosa_config *c, const nosa_state *st, const uint16_t *q, void *split,
+                         size_t split_bytes, void *ws, size_t ws_bytes, void *stream) {
+    return run_decode(c, st, q, kModeResident, nullptr, nullptr, nullptr, nullptr, split, split_bytes, nullptr,
+                      ws, ws_bytes, stream);
+}
+
+int nosa_decode_rest(const nosa_config *c, const nosa_state *st, const uint16_t *q, const int32_t *gq,
+                     const void *split, size_t split_bytes, uint16_t *out, void *ws, size_t ws_bytes,
+                     void *stream) {
+    return run_decode(c, st, q, kModeRest, nullptr, nullptr, nullptr, gq, const_cast<void *>(split), split_bytes,
+                      out, ws, ws_bytes, stream);
 }
 
 int nosa_dense_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q,
                       uint16_t *out, void *ws, size_t ws_bytes, void *stream) {
     if (c && c->offload) return NOSA_ERR_ARG;
-    return run_decode(c, st, q, nullptr, nullptr, nullptr, out, ws, ws_bytes, stream, true);
+    return run_decode(c, st, q, kModeDense, nullptr, nullptr, nullptr, nullptr, nullptr, 0, out, ws, ws_bytes,
+                      stream);
 }
 
 int nosa_read_error(const nosa_state *st, uint32_t *flags, int clear, void *stream) {

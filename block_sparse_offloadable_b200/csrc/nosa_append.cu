@@ -454,7 +454,13 @@ __global__ void __launch_bounds__(256) prefill_gamma_kernel(const AppendParams p
         int32_t at = pre - cnt;
         int32_t *ge = p.gamma_e + (int64_t)u * p.k_e;
         for (int i = b0; i < b1; ++i)
-            if (flag[i]) ge[at++] = i;
+            if (flag[i]) {
+                if (p.offload) {  // Gamma_e starts resident: slot 1 + its place in the ascending list
+                    p.slot_block[(int64_t)u * p.nslots + 1 + at] = i;
+                    p.block_slot[(int64_t)u * p.nblk + i] = 1 + at;
+                }
+                ge[at++] = i;
+            }
         if (lane == 31) {
             p.gamma_n[u] = pre;
             if (p.offload && len > 0) {
@@ -463,6 +469,26 @@ __global__ void __launch_bounds__(256) prefill_gamma_kernel(const AppendParams p
                 p.block_slot[(int64_t)u * p.nblk + local] = 0;
             }
             p.seq_len[u] = len;
+        }
+    }
+    if (p.offload) {
+        // copy the Gamma_e blocks from the prefill input (on the device) into their
+        // cache slots: the first decode step then finds Gamma_e resident, as every
+        // later step does (Gamma_e(t) lies in S(t-1) plus the previous local block)
+        __syncthreads();
+        const int32_t n = min(p.gamma_n[u], p.k_e);
+        const int32_t *ge = p.gamma_e + (int64_t)u * p.k_e;
+        constexpr int kChunks = kBlockBytes / 16, kHalfChunks = kHalfBlockBytes / 16, kRowChunks = kRowBytes / 16;
+        for (int j = 0; j < n; ++j) {
+            const int32_t b = ge[j];
+            uint4 *dst = reinterpret_cast<uint4 *>(p.cache + ((int64_t)u * p.nslots + 1 + j) * kBlockBytes);
+            for (int c = threadIdx.x; c < kChunks; c += blockDim.x) {
+                const int half = c / kHalfChunks, rem = c % kHalfChunks;
+                const int row = rem / kRowChunks, col = rem % kRowChunks;
+                const uint16_t *src =
+                    (half ? p.v_new : p.k_new) + ((int64_t)u * p.T + (int64_t)b * kBlock + row) * kD;
+                dst[c] = reinterpret_cast<const uint4 *>(src)[col];
+            }
         }
     }
 }

@@ -47,8 +47,13 @@ namespace {
 constexpr int kDecW = 4;                  // warps per consumer group (16 tokens of a block each)
 constexpr int kGroups = 2;                // consumer groups, taking alternate blocks
 constexpr int kConsWarps = kDecW * kGroups;
-constexpr int kDecS = 6;                  // ring stages (one block each); one CTA per SM
-static_assert(kDecS % kGroups == 0, "stage s must always be consumed by group s % kGroups");
+// Ring stages (one block each; one CTA per SM).  The resident pass of the
+// split decode uses fewer, so that one of its CTAs and one select CTA fit on an
+// SM together and the two kernels really run concurrently.
+constexpr int kDecS = 6;
+constexpr int kDecSResident = 4;
+static_assert(kDecS % kGroups == 0 && kDecSResident % kGroups == 0,
+              "stage s must always be consumed by group s % kGroups");
 constexpr int kBoxBytes = 64 * 128;       // one TMA box: 64 rows x 64 bf16
 constexpr int kDecThreads = (kConsWarps + 1) * 32;
 constexpr int kConsThreads = kConsWarps * 32;
@@ -63,12 +68,53 @@ __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsThreads) : "memory");
 }
 
-// Work items of unit u: its selected blocks (sparse) or all its blocks (dense).
+// Work items of unit u in the kernel's mode.
 __device__ __forceinline__ int32_t unit_work(const DecodeParams &p, int32_t u) {
     const int32_t L = p.seq_len[u];
     if (L <= 0) return 0;
-    if (p.sel) return max(0, min(p.nsel[u], p.max_sel));
-    return (L + kBlock - 1) / kBlock;
+    switch (p.mode) {
+    case kModeSel: return max(0, min(p.nsel[u], p.max_sel));
+    case kModeResident: return min(max(p.gamma_n[u], 0), p.k_e) + 1;
+    case kModeRest: return p.k_q;
+    default: return (L + kBlock - 1) / kBlock;
+    }
+}
+
+// Block id (lb; -1 = nothing to attend) and buffer block index (pb) of item j of unit u.
+__device__ __forceinline__ void item_block(const DecodeParams &p, int32_t u, int32_t j, int32_t &lb, int32_t &pb) {
+    if (p.mode == kModeSel) {
+        lb = p.sel[(int64_t)u * p.max_sel + j];
+        pb = p.block_table ? p.block_table[(int64_t)u * p.max_sel + j] : lb;
+        return;
+    }
+    if (p.mode == kModeDense) {
+        lb = pb = j;
+        return;
+    }
+    if (p.mode == kModeResident) {
+        const int32_t ne = min(max(p.gamma_n[u], 0), p.k_e);
+        lb = (j < ne) ? p.gamma_e[(int64_t)u * p.k_e + j] : (p.seq_len[u] - 1) / kBlock;
+    } else {  // kModeRest: Gamma_q entries not already attended by the resident pass
+        lb = p.gq[(int64_t)u * p.k_q + j];
+        if (lb >= 0 && lb < p.nblk &&
+            ((p.res_bits[(int64_t)u * p.bits_words + (lb >> 5)] >> (lb & 31)) & 1u))
+            lb = -1;
+    }
+    pb = (p.block_slot && lb >= 0 && lb < p.nblk) ? p.block_slot[(int64_t)u * p.nblk + lb] : lb;
+}
+
+// Merge the resident pass's state of unit u (head h, dim d) into (M, acc, lsum) in place.
+__device__ __forceinline__ void merge_resident(const DecodeParams &p, int32_t u, int h, int d, float &M, float &acc,
+                                               float &lsum) {
+    const float *r = p.res_part + (int64_t)u * kPartFloats;
+    const float rm = r[h];
+    const float Mn = fmaxf(M, rm);
+    if (Mn == -__builtin_huge_valf()) return;
+    const float fa = (M == -__builtin_huge_valf()) ? 0.f : exp2f(M - Mn);
+    const float fr = (rm == -__builtin_huge_valf()) ? 0.f : exp2f(rm - Mn);
+    acc = fmaf(fr, r[2 * kMaxG + h * kD + d], fa * acc);
+    lsum = fmaf(fr, r[kMaxG + h], fa * lsum);
+    M = Mn;
 }
 
 // Largest u with P[u] <= x, for 0 <= x < P[U] (skips units without work).
@@ -196,14 +242,15 @@ __device__ __forceinline__ void store_bf16(uint16_t *dst, float v) {
 }
 }  // namespace
 
-size_t decode_smem_bytes(int32_t units) {
-    return 1024 + (size_t)kDecS * kBlockBytes + (size_t)kDecS * kBlock * sizeof(float) +
-           2 * kDecS * sizeof(uint64_t) + kDecS * sizeof(int32_t) + (size_t)kDecW * kPartFloats * sizeof(float) +
+size_t decode_smem_bytes(int32_t units, int stages) {
+    return 1024 + (size_t)stages * kBlockBytes + (size_t)stages * kBlock * sizeof(float) +
+           2 * stages * sizeof(uint64_t) + stages * sizeof(int32_t) + (size_t)kDecW * kPartFloats * sizeof(float) +
            ((size_t)units + 1) * sizeof(int32_t);
 }
 
 int decode_ctas() { return kNumSms; }
 
+template <int kStages>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p) {
     pdl_trigger();  // the next append's CTAs are tiny; they wait for this grid
@@ -211,11 +258,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *tiles = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float *ebuf = reinterpret_cast<float *>(tiles + kDecS * kBlockBytes);
-    uint64_t *full = reinterpret_cast<uint64_t *>(ebuf + kDecS * kBlock);
-    uint64_t *empty = full + kDecS;
-    int32_t *s_blk = reinterpret_cast<int32_t *>(empty + kDecS);
-    float *scratch = reinterpret_cast<float *>(s_blk + kDecS);
+    float *ebuf = reinterpret_cast<float *>(tiles + kStages * kBlockBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(ebuf + kStages * kBlock);
+    uint64_t *empty = full + kStages;
+    int32_t *s_blk = reinterpret_cast<int32_t *>(empty + kStages);
+    float *scratch = reinterpret_cast<float *>(s_blk + kStages);
     int32_t *P = reinterpret_cast<int32_t *>(scratch + kDecW * kPartFloats);
     __shared__ int32_t s_wsum[kConsWarps + 1];
     __shared__ int s_last;
@@ -225,7 +272,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int32_t U = p.units, G = (int32_t)gridDim.x, cta = (int32_t)blockIdx.x;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kDecS; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kDecW);
         }
@@ -276,22 +323,21 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             if (lane < nb) {
                 const int64_t x = xb + lane;
                 bu = find_unit(P, U, x);
-                const int32_t j = (int32_t)(x - P[bu]);
-                blb = p.sel ? p.sel[(int64_t)bu * p.max_sel + j] : j;
-                bpb = p.block_table ? p.block_table[(int64_t)bu * p.max_sel + j] : blb;
+                item_block(p, bu, (int32_t)(x - P[bu]), blb, bpb);
             }
             for (int k = 0; k < nb; ++k, ++it) {
                 const int32_t u = __shfl_sync(0xFFFFFFFFu, bu, k);
                 const int32_t lb = __shfl_sync(0xFFFFFFFFu, blb, k);
                 const int32_t pb = __shfl_sync(0xFFFFFFFFu, bpb, k);
                 if (lane == 0) {
-                    const int s = it % kDecS;
+                    const int s = it % kStages;
                     const bool go =
-                        it < kDecS || wait_or_abort(&empty[s], ((it / kDecS) - 1) & 1, &s_abort, p.err);
+                        it < kStages || wait_or_abort(&empty[s], ((it / kStages) - 1) & 1, &s_abort, p.err);
                     if (go) {
                         const bool ok = lb >= 0 && (int64_t)lb * kBlock < p.max_ctx && pb >= 0 &&
                                         pb < p.blocks_per_unit;
                         s_blk[s] = ok ? lb : -1;
+                        if (!ok && lb >= 0) set_error(p.err, NOSA_EFLAG_STATE);  // a block with no buffer
                         if (ok) {
                             const int32_t y = (int32_t)(((int64_t)u * p.blocks_per_unit + pb) * 2 * kBlock);
                             uint8_t *t = tiles + s * kBlockBytes;
@@ -313,7 +359,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
         // never leave with copies in flight
         if (lane == 0)
-            for (int i = max(0, it - kDecS); i < it; ++i) mbar_wait(&full[i % kDecS], (i / kDecS) & 1);
+            for (int i = max(0, it - kStages); i < it; ++i) mbar_wait(&full[i % kStages], (i / kStages) & 1);
     } else {
         // ---------------- consumers ----------------
         // Group g takes the CTA's items of parity g (stage s = item % 6 is always
@@ -346,8 +392,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             const int slot = (u == first_unit) ? 0 : 1;
             for (int64_t xi = x + ((((x - lo) & 1) != grp) ? 1 : 0); xi < seg_end; xi += kGroups) {
                 const int it = (int)(xi - lo);
-                const int s = it % kDecS;
-                if (wait_or_abort(&full[s], (it / kDecS) & 1, &s_abort, p.err)) {
+                const int s = it % kStages;
+                if (wait_or_abort(&full[s], (it / kStages) & 1, &s_abort, p.err)) {
                     const int32_t lb = s_blk[s];
                     if (lb >= 0)
                         attend_block(st, qf, tiles + s * kBlockBytes, ebuf + s * kBlock, lb, L, p.qk_log2,
@@ -432,7 +478,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     acc = fmaf(f, scratch[w * kPartFloats + 2 * kMaxG + h * kD + d], acc);
                     lsum = fmaf(f, scratch[w * kPartFloats + kMaxG + h], lsum);
                 }
-                if (whole) {
+                if (whole && p.mode == kModeResident) {
+                    float *rp = p.res_part + (int64_t)u * kPartFloats;
+                    rp[2 * kMaxG + h * kD + d] = acc;
+                    if (d == 0) {
+                        rp[h] = M;
+                        rp[kMaxG + h] = lsum;
+                    }
+                } else if (whole) {
+                    if (p.mode == kModeRest) merge_resident(p, u, h, d, M, acc, lsum);
                     store_bf16(out + idx, lsum > 0.f ? acc / lsum : 0.f);
                 } else {
                     part[2 * kMaxG + h * kD + d] = acc;
@@ -452,31 +506,41 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     // last contributor: merge the unit's partials in CTA order
                     __threadfence();
                     if (ctid == 0) p.counter[u] = 0;
-                    const int nc = cl - cf + 1;                         // <= Ge <= number of CTAs
+                    // the CTA partials (and, merging the rest pass, the resident state)
+                    const int nc = cl - cf + 1 + (p.mode == kModeRest ? 1 : 0);  // <= Ge + 1
                     float *fac = scratch;                               // [nc][8] scale of each partial
                     float *lsum = fac + nc * kMaxG;                     // [8] merged denominators
-                    int32_t *offs = reinterpret_cast<int32_t *>(lsum + kMaxG);  // [nc] partial offsets
+                    float *Ms = lsum + kMaxG;                           // [8] merged maxima
+                    const float **src = reinterpret_cast<const float **>(
+                        scratch + ((nc * kMaxG + 2 * kMaxG + 1) & ~1));  // [nc] partial states
                     for (int t = ctid; t < nc; t += kConsThreads) {
                         const int32_t cc = cf + t;
-                        const int sl = (find_unit(P, U, (int64_t)cc * W / Ge) == u) ? 0 : 1;
-                        offs[t] = (cc * 2 + sl) * kPartFloats;
+                        if (cc > cl) {
+                            src[t] = p.res_part + (int64_t)u * kPartFloats;
+                        } else {
+                            const int sl = (find_unit(P, U, (int64_t)cc * W / Ge) == u) ? 0 : 1;
+                            src[t] = p.part + (int64_t)(cc * 2 + sl) * kPartFloats;
+                        }
                     }
                     consumer_sync();
                     for (int h = warp; h < p.G; h += kConsWarps) {  // one warp per head
                         float M = kNegInf;
-                        for (int t = lane; t < nc; t += 32) M = fmaxf(M, __ldcg(p.part + offs[t] + h));
+                        for (int t = lane; t < nc; t += 32) M = fmaxf(M, __ldcg(src[t] + h));
 #pragma unroll
                         for (int sh = 16; sh > 0; sh >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, sh));
                         float ls = 0.f;
                         for (int t = lane; t < nc; t += 32) {
-                            const float mc = __ldcg(p.part + offs[t] + h);
+                            const float mc = __ldcg(src[t] + h);
                             const float f = (mc == kNegInf) ? 0.f : exp2f(mc - M);
                             fac[t * kMaxG + h] = f;
-                            ls = fmaf(f, __ldcg(p.part + offs[t] + kMaxG + h), ls);
+                            ls = fmaf(f, __ldcg(src[t] + kMaxG + h), ls);
                         }
 #pragma unroll
                         for (int sh = 16; sh > 0; sh >>= 1) ls += __shfl_xor_sync(0xFFFFFFFFu, ls, sh);
-                        if (lane == 0) lsum[h] = ls;
+                        if (lane == 0) {
+                            lsum[h] = ls;
+                            Ms[h] = M;
+                        }
                     }
                     consumer_sync();
                     for (int v = ctid; v < p.G * (kD / 4); v += kConsThreads) {  // 4 dims per thread
@@ -485,12 +549,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll 4
                         for (int t = 0; t < nc; ++t) {
                             const float f = fac[t * kMaxG + h];
-                            const float4 o4 = __ldcg(reinterpret_cast<const float4 *>(
-                                p.part + offs[t] + 2 * kMaxG + h * kD + d4));
+                            const float4 o4 = __ldcg(reinterpret_cast<const float4 *>(src[t] + 2 * kMaxG + h * kD + d4));
                             acc.x = fmaf(f, o4.x, acc.x); acc.y = fmaf(f, o4.y, acc.y);
                             acc.z = fmaf(f, o4.z, acc.z); acc.w = fmaf(f, o4.w, acc.w);
                         }
                         const float ls = lsum[h];
+                        if (p.mode == kModeResident) {  // the unit's state, for the rest pass
+                            float *rp = p.res_part + (int64_t)u * kPartFloats;
+                            *reinterpret_cast<float4 *>(rp + 2 * kMaxG + h * kD + d4) = acc;
+                            if (d4 == 0) {
+                                rp[h] = Ms[h];
+                                rp[kMaxG + h] = ls;
+                            }
+                            continue;
+                        }
                         uint2 pk;
                         if (ls > 0.f) {
                             pk.x = pack_bf16x2(acc.x / ls, acc.y / ls);
@@ -507,24 +579,54 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             x = seg_end;
             u = u_next;
         }
-        // units without work (no tokens): zero output, one CTA each
+        // units without work, one CTA each: zero output (an empty state in the
+        // resident pass; the resident state alone in the rest pass)
         for (int32_t uz = cta; uz < U; uz += G) {
             if (P[uz + 1] != P[uz]) continue;
+            if (p.mode == kModeResident) {
+                float *rp = p.res_part + (int64_t)uz * kPartFloats;
+                for (int i = ctid; i < kPartFloats; i += kConsThreads) rp[i] = (i < kMaxG) ? kNegInf : 0.f;
+                continue;
+            }
             uint16_t *out = p.out + (int64_t)uz * p.G * kD;
-            for (int idx = ctid; idx < p.G * kD; idx += kConsThreads) out[idx] = 0;
+            for (int idx = ctid; idx < p.G * kD; idx += kConsThreads) {
+                float M = kNegInf, acc = 0.f, lsum = 0.f;
+                if (p.mode == kModeRest) merge_resident(p, uz, idx >> 7, idx & (kD - 1), M, acc, lsum);
+                store_bf16(out + idx, lsum > 0.f ? acc / lsum : 0.f);
+            }
+        }
+        // the resident pass also leaves, per unit, the set it covered (for the rest pass)
+        if (p.mode == kModeResident) {
+            for (int32_t uz = cta; uz < U; uz += G) {
+                uint32_t *bits = p.res_bits + (int64_t)uz * p.bits_words;
+                for (int i = ctid; i < p.bits_words; i += kConsThreads) bits[i] = 0u;
+                consumer_sync();
+                const int32_t Lz = p.seq_len[uz];
+                const int32_t ne = Lz > 0 ? min(max(p.gamma_n[uz], 0), p.k_e) : -1;
+                for (int j = ctid; j <= ne; j += kConsThreads) {
+                    const int32_t b = (j < ne) ? p.gamma_e[(int64_t)uz * p.k_e + j] : (Lz - 1) / kBlock;
+                    if (b >= 0 && b < p.nblk) atomicOr(&bits[b >> 5], 1u << (b & 31));
+                }
+            }
         }
     }
 }
 
-int launch_decode(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t stream) {
-    const size_t smem = decode_smem_bytes(p.units);
-    if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+template <int kStages>
+int launch_decode_t(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t stream) {
+    const size_t smem = decode_smem_bytes(p.units, kStages);
+    if (cudaFuncSetAttribute(decode_kernel<kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
         return NOSA_ERR_CUDA;
-    return launch_pdl(decode_kernel, dim3(decode_ctas()), dim3(kDecThreads), smem, stream, tmap, p) ==
+    return launch_pdl(decode_kernel<kStages>, dim3(decode_ctas()), dim3(kDecThreads), smem, stream, tmap, p) ==
                    cudaSuccess
                ? NOSA_OK
                : NOSA_ERR_CUDA;
+}
+
+int launch_decode(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t stream) {
+    return p.mode == kModeResident ? launch_decode_t<kDecSResident>(p, tmap, stream)
+                                   : launch_decode_t<kDecS>(p, tmap, stream);
 }
 
 }  // namespace nosa

@@ -67,9 +67,15 @@ struct CacheParams {
     int32_t nblk, nslots, units, max_sel;
 };
 
+// Work lists of the decode kernel.
+constexpr int kModeSel = 0;       // the blocks of S(t) (sel / nsel)
+constexpr int kModeDense = 1;     // every block (the dense comparator)
+constexpr int kModeResident = 2;  // Gamma_e + the local block, known right after the append
+constexpr int kModeRest = 3;      // the blocks of Gamma_q outside Gamma_e + local, merged with the above
+
 struct DecodeParams {
     const uint16_t *q;          // [B][Hq][D]
-    const int32_t *sel;         // [u][max_sel], or null = every block (dense)
+    const int32_t *sel;         // [u][max_sel] (kModeSel)
     const int32_t *nsel;        // [u]
     const int32_t *block_table; // [u][max_sel] or null (block id addresses the store)
     const float *e;             // [u][max_ctx]
@@ -82,6 +88,14 @@ struct DecodeParams {
     int32_t blocks_per_unit;    // blocks per unit in the tensor-mapped buffer (nblk or nslots)
     int32_t max_sel, G, units;
     float qk_log2;              // scale * log2(e)
+    int32_t mode;
+    const int32_t *gamma_e;     // kModeResident: [u][k_e] ascending, and gamma_n [u]
+    const int32_t *gamma_n;
+    const int32_t *gq;          // kModeRest: [u][k_q] Gamma_q, -1 padded
+    const int32_t *block_slot;  // kModeResident / kModeRest with offload: [u][nblk] cache slot, else null
+    float *res_part;            // [u][kPartFloats] state over Gamma_e + local (written by resident, read by rest)
+    uint32_t *res_bits;         // [u][bits_words] membership of Gamma_e + local (same)
+    int32_t k_e, k_q, nblk, bits_words;
 };
 
 constexpr int kPartFloats = 2 * kMaxG + kMaxG * kD;  // m[8], l[8], o[8][128]

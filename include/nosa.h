@@ -55,7 +55,8 @@ extern "C" {
 #define NOSA_EFLAG_CAPACITY 0x1u   /* append beyond max_ctx: token dropped */
 #define NOSA_EFLAG_TIMEOUT 0x2u    /* a bounded mbarrier wait gave up: output of that tile invalid */
 #define NOSA_EFLAG_NOSLOT 0x4u     /* offload cache had no free slot: token dropped */
-#define NOSA_EFLAG_STATE 0x8u      /* state inconsistent (prefill into a non-empty unit, lost local block) */
+#define NOSA_EFLAG_STATE 0x8u      /* state inconsistent (prefill into a non-empty unit, lost local block,
+                                       a block to attend that has no cache slot) */
 
 /*
  * Problem configuration.  Built: head_dim 128, block 64, sub_block 16,
@@ -157,7 +158,8 @@ enum nosa_call {
     NOSA_WS_SELECT = 0,
     NOSA_WS_SPARSE_DECODE = 1,
     NOSA_WS_DENSE_DECODE = 2,
-    NOSA_WS_CACHE_SYNC = 3
+    NOSA_WS_CACHE_SYNC = 3,
+    NOSA_WS_SPLIT = 4  /* the buffer nosa_decode_resident fills and nosa_decode_rest reads */
 };
 
 /* Validate a configuration: NOSA_OK or a negative code. */
@@ -202,7 +204,8 @@ int nosa_state_init(const nosa_config *cfg, const nosa_state *st, void *stream);
  * rank, and nosa_select forms Gamma_e.  Prefill builds the pooled arrays and
  * Gamma_e = top-k_e by E (ties to the lower block), with NOSA_FLAG_FILL the
  * pool of every candidate in rank order, and, in offload mode, puts the local
- * block in the cache.
+ * block and the Gamma_e blocks in the cache (from the prefill input, without a
+ * host transfer), so that Gamma_e is resident from the first decode step on.
  * Device errors: NOSA_EFLAG_CAPACITY (L + T > max_ctx; unit skipped),
  * NOSA_EFLAG_STATE (prefill into a non-empty unit), NOSA_EFLAG_NOSLOT.
  */
@@ -308,6 +311,37 @@ int nosa_sparse_decode(const nosa_config *cfg, const nosa_state *st, const uint1
  */
 int nosa_dense_decode(const nosa_config *cfg, const nosa_state *st, const uint16_t *q,
                       uint16_t *out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * a5 split in two, so that the blocks already on the GPU are attended while
+ * the missed ones are fetched.  NOSA pages: montaan.com summary of
+ * 2510.13602, "Empirical Results and Analysis" item 4 (the wall-time
+ * breakdown: decoding is bound by KV loading) and "System Optimization
+ * (NOSI)" item 2 (only blocks unused in the current step are swapped out).
+ * Union reading only (NOSA_ERR_UNSUPPORTED with NOSA_FLAG_FILL, where Gamma_e
+ * depends on Gamma_q).
+ *
+ * nosa_decode_resident: right after nosa_compress_append of the step, and
+ * concurrently with nosa_select / nosa_cache_sync (another stream).  Attends
+ * over R(t) = Gamma_e(t) + {local block} as left by the append; every block of
+ * R(t) is on the GPU already (Gamma_e(t) lies in S(t-1) plus the previous
+ * local block, and a cache sync never frees a block of S(t)).  Writes into
+ * `split` (nosa_workspace_bytes(cfg, NOSA_WS_SPLIT) bytes, device) each unit's
+ * softmax state over R(t) and the set R(t).
+ *
+ * nosa_decode_rest: after nosa_select (its gq output), nosa_cache_sync and
+ * nosa_decode_resident.  Attends over Gamma_q(t) minus R(t), merges with the
+ * state in `split`, and writes `out` exactly as nosa_sparse_decode would (up
+ * to the order of floating-point sums).
+ *
+ *   ws  device workspace of nosa_workspace_bytes(cfg, NOSA_WS_SPARSE_DECODE) bytes each;
+ *       the two calls may share one, as they never overlap
+ */
+int nosa_decode_resident(const nosa_config *cfg, const nosa_state *st, const uint16_t *q, void *split,
+                         size_t split_bytes, void *ws, size_t ws_bytes, void *stream);
+int nosa_decode_rest(const nosa_config *cfg, const nosa_state *st, const uint16_t *q, const int32_t *gq,
+                     const void *split, size_t split_bytes, uint16_t *out, void *ws, size_t ws_bytes,
+                     void *stream);
 
 /*
  * Read the device error word (synchronises the stream).  *flags receives the

@@ -28,7 +28,7 @@ MAX_ABS, MEAN_ABS, REL_L2 = 1e-2, 1e-3, 1e-2
 
 class Scenario:
     def __init__(self, B, Hq, Hkv, k_q, k_e, L0, steps, offload=False, seed=0, layer=0, lens=None,
-                 max_ctx=None, dense=False, ck_bf16=False, fill=False, head=False):
+                 max_ctx=None, dense=False, ck_bf16=False, fill=False, head=False, split=False):
         self.B, self.Hq, self.Hkv, self.k_q, self.k_e = B, Hq, Hkv, k_q, k_e
         self.G = Hq // Hkv
         self.units = B * Hkv
@@ -40,6 +40,7 @@ class Scenario:
         self.ck_bf16 = ck_bf16
         self.fill = fill
         self.head = head  # eviction logits from the fused head (synthetic weights) instead of inputs
+        self.split = split  # decode_resident on a side stream during select / cache_sync, then decode_rest
         self.W = synth.head_weights(seed, layer, Hkv) if head else None
 
     def cfg(self):
@@ -100,6 +101,7 @@ def run_gpu(sc, data):
         append(_dev16(kp), _dev16(vp), torch.from_numpy(ep).cuda(), T,
                torch.from_numpy(lens).cuda() if ragged else None)
     res = {k: [] for k in ("sel", "nsel", "gq", "ge", "gn", "out", "nf", "dense")}
+    side = torch.cuda.Stream() if sc.split else None
     for t in range(sc.steps):
         idx = lens.repeat(sc.Hkv) + t  # position of this step's token, per unit
         kn = _dev16(K[np.arange(sc.units), idx][:, None, :])
@@ -108,10 +110,18 @@ def run_gpu(sc, data):
         q = _dev16(Q[t])
         out = torch.empty((sc.B, sc.Hq, 128), dtype=torch.int16, device="cuda")
         append(kn, vn, en, 1)
+        if sc.split:
+            cur = torch.cuda.current_stream()
+            side.wait_stream(cur)
+            lay.decode_resident(q, side)
         lay.select(q)
         if sc.offload:
             lay.cache_sync()
-        lay.sparse_decode(q, out)
+        if sc.split:
+            cur.wait_stream(side)
+            lay.decode_rest(q, out)
+        else:
+            lay.sparse_decode(q, out)
         res["sel"].append(lay.sel.cpu().numpy())
         res["nsel"].append(lay.nsel.cpu().numpy())
         res["gq"].append(lay.gq.cpu().numpy())
