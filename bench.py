@@ -449,6 +449,49 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
+# DRAM bytes per launch from an ncu capture (profiles/dram_traffic.json): used only for the
+# same workload variant and only while the kernel's sources are unchanged since the capture.
+KERNEL_SOURCES = {
+    "select": "nosa_select.cu", "decode": "nosa_decode.cu", "cache_sync": "nosa_cache.cu",
+    "append": "nosa_append.cu",
+}
+
+
+def sources_sha(name):
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_offloadable_b200", "csrc")
+    for f in (KERNEL_SOURCES[name], "nosa_common.cuh", "nosa_internal.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def captured_traffic(name, variant):
+    """(bytes per launch, capture note) for kernel `name` on `variant`, or (None, why not)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            table = json.load(f)
+    except (OSError, ValueError):
+        return None, "no capture"
+    for e in table.get("captures", []):
+        if e.get("kernel") == name and e.get("variant") == variant:
+            if e.get("sources_sha256") != sources_sha(name):
+                return None, "kernel changed since the capture"
+            return float(e["dram_bytes_per_launch"]), e.get("profile")
+    return None, "no capture of this variant"
+
+
+def traffic_variant(c, args):
+    """The workload variant a traffic capture must match: the workload name plus the options that change
+    the kernels' work (the layer count does not change a launch)."""
+    v = [args.workload]
+    for key in ("ck_bf16", "fill", "head", "split"):
+        if c.get(key):
+            v.append(key)
+    return "+".join(v)
+
+
 # ---------------------------------------------------------------------------------------
 
 def oracle_sample(c, groups, seed, n_units, n_steps, budget_s=25.0):
@@ -654,6 +697,11 @@ def run_nosa(args, c, rank, world, dev):
     hb = max((k for k in kern if "frac_hbm" in kern[k]), key=lambda k: kern[k]["share"])
     roof_hbm = {"bound": "hbm", "kernel": hb, "achieved": kern[hb]["GBps"], "peak": hbm_peak, "unit": "GB/s",
                 "frac": kern[hb]["frac_hbm"], "traffic": None}
+    variant = traffic_variant(c, args)
+    for r in (roof, roof_hbm):
+        kname = "cache_sync" if r["kernel"].startswith("cache_sync") else r["kernel"]
+        if kname in KERNEL_SOURCES:
+            r["traffic"], r["traffic_source"] = captured_traffic(kname, variant)
 
     # ---- end to end: host inputs -> device, step, outputs -> host, all inside the timed region ----
     e2e = None
