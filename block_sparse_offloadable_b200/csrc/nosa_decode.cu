@@ -7,10 +7,13 @@
 //
 // Design: persistent split-K flash decoding with GQA sharing.
 //  * Work items are (unit, selected block) pairs, unit = (seq, kv head).  Each
-//    CTA (one per SM) computes the prefix sum of the per-unit item counts (from
-//    nsel, or from seq_len for the dense comparator) in shared memory and takes
-//    an exactly balanced contiguous range of the flattened item list, so every
-//    SM streams the same number of 32 KiB blocks whatever the unit count.
+//    CTA (one per SM) holds the item offsets of the units in shared memory and
+//    takes an exactly balanced contiguous range of the flattened item list, so
+//    every SM streams the same number of 32 KiB blocks whatever the unit count.
+//    The sparse decode gives every unit max_sel items (nsel is max_sel or just
+//    below it once the context holds k blocks; the -1 padding past nsel is
+//    skipped), which spares a round of global reads before the first block-id
+//    load; the other work lists count their items with a prefix sum.
 //  * One producer thread streams the range's blocks (keys + values, plus the
 //    64 eviction logits) into a 6-stage shared-memory ring: four 2-D TMA tile
 //    loads (64 rows x 64 dims, 128-byte swizzle) and one bulk copy per block,
@@ -29,7 +32,9 @@
 //    more m16n8k16 tiles whose A fragments are built from 16-byte value loads
 //    with byte permutes (output dims permuted, undone at the store).
 //  * A CTA's range splits into unit segments.  At a segment's end the four
-//    warps merge their (m, l, o) states in shared memory (named barrier, the
+//    warps merge their (m, l, o) states in shared memory (a padded, swizzled
+//    layout that spreads each warp's fragment-order stores over 32 banks; named
+//    barrier, the
 //    producer keeps streaming); a segment covering its whole unit writes bf16
 //    output, otherwise the partial state goes to the CTA's workspace slot (only
 //    a CTA's first and last segments can be partial) and the last of the
@@ -59,6 +64,11 @@ constexpr int kDecThreads = (kConsWarps + 1) * 32;
 constexpr int kConsThreads = kConsWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kNegInf = -__builtin_huge_valf();
+// Merge scratch per warp: m[8], l[8], o[8][kHS] with a padded head row and bit 0 of the
+// dim XOR-ed with bit 5, so the fragment-order stores of a warp hit 32 distinct banks.
+constexpr int kHS = kD + 1;
+constexpr int kScr = 2 * kMaxG + kMaxG * kHS;
+__device__ __forceinline__ int swz(int x) { return x ^ ((x >> 5) & 1); }
 
 __device__ __forceinline__ uint32_t word(const uint4 &v, int i) {
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
@@ -244,7 +254,7 @@ __device__ __forceinline__ void store_bf16(uint16_t *dst, float v) {
 
 size_t decode_smem_bytes(int32_t units, int stages) {
     return 1024 + (size_t)stages * kBlockBytes + (size_t)stages * kBlock * sizeof(float) +
-           2 * stages * sizeof(uint64_t) + stages * sizeof(int32_t) + (size_t)kDecW * kPartFloats * sizeof(float) +
+           2 * stages * sizeof(uint64_t) + stages * sizeof(int32_t) + (size_t)kDecW * kScr * sizeof(float) +
            ((size_t)units + 1) * sizeof(int32_t);
 }
 
@@ -263,7 +273,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     uint64_t *empty = full + kStages;
     int32_t *s_blk = reinterpret_cast<int32_t *>(empty + kStages);
     float *scratch = reinterpret_cast<float *>(s_blk + kStages);
-    int32_t *P = reinterpret_cast<int32_t *>(scratch + kDecW * kPartFloats);
+    int32_t *P = reinterpret_cast<int32_t *>(scratch + kDecW * kScr);
     __shared__ int32_t s_wsum[kConsWarps + 1];
     __shared__ int s_last;
     __shared__ volatile int s_abort;
@@ -280,8 +290,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         prefetch_tmap(&tmap);
         s_abort = 0;
     }
-    // ---- prefix sum of the per-unit work: P[u] = items of units < u ----
-    {
+    // ---- P[u] = items of units < u ----
+    if (p.mode == kModeSel) {
+        // nominal ranges: max_sel items per unit, whatever nsel (sel is -1 padded past nsel,
+        // and such items are skipped); no global read stands before the first block-id load
+        for (int u = threadIdx.x; u <= U; u += blockDim.x) P[u] = u * p.max_sel;
+    } else {  // prefix sum of the per-unit work
         const int per = (U + kDecThreads - 1) / kDecThreads;
         const int u0 = min((int)threadIdx.x * per, U), u1 = min(u0 + per, U);
         int32_t sum = 0;
@@ -411,7 +425,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, sh);
                 l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, sh);
             }
-            float *mine = scratch + wq * kPartFloats;
+            float *mine = scratch + wq * kScr;
             float *oo = mine + 2 * kMaxG;
             if (grp == 0) {
                 if (r == 0) {
@@ -421,10 +435,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
                 for (int t = 0; t < 8; ++t) {
                     const int psi = 64 * (t >> 2) + 8 * sig + 2 * (t & 3);
-                    oo[(2 * c) * kD + psi] = st.o[t][0];
-                    oo[(2 * c + 1) * kD + psi] = st.o[t][1];
-                    oo[(2 * c) * kD + psi + 1] = st.o[t][2];
-                    oo[(2 * c + 1) * kD + psi + 1] = st.o[t][3];
+                    oo[(2 * c) * kHS + swz(psi)] = st.o[t][0];
+                    oo[(2 * c + 1) * kHS + swz(psi)] = st.o[t][1];
+                    oo[(2 * c) * kHS + swz(psi + 1)] = st.o[t][2];
+                    oo[(2 * c + 1) * kHS + swz(psi + 1)] = st.o[t][3];
                 }
             }
             consumer_sync();
@@ -440,10 +454,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
                 for (int t = 0; t < 8; ++t) {
                     const int psi = 64 * (t >> 2) + 8 * sig + 2 * (t & 3);
-                    om[t][0] = fmaf(fa0, oo[(2 * c) * kD + psi], fb0 * st.o[t][0]);
-                    om[t][1] = fmaf(fa1, oo[(2 * c + 1) * kD + psi], fb1 * st.o[t][1]);
-                    om[t][2] = fmaf(fa0, oo[(2 * c) * kD + psi + 1], fb0 * st.o[t][2]);
-                    om[t][3] = fmaf(fa1, oo[(2 * c + 1) * kD + psi + 1], fb1 * st.o[t][3]);
+                    om[t][0] = fmaf(fa0, oo[(2 * c) * kHS + swz(psi)], fb0 * st.o[t][0]);
+                    om[t][1] = fmaf(fa1, oo[(2 * c + 1) * kHS + swz(psi)], fb1 * st.o[t][1]);
+                    om[t][2] = fmaf(fa0, oo[(2 * c) * kHS + swz(psi + 1)], fb0 * st.o[t][2]);
+                    om[t][3] = fmaf(fa1, oo[(2 * c + 1) * kHS + swz(psi + 1)], fb1 * st.o[t][3]);
                 }
                 __syncwarp();  // every lane has read m, l before lanes r == 0 overwrite them
                 if (r == 0) {
@@ -454,10 +468,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
                 for (int t = 0; t < 8; ++t) {
                     const int psi = 64 * (t >> 2) + 8 * sig + 2 * (t & 3);
-                    oo[(2 * c) * kD + psi] = om[t][0];
-                    oo[(2 * c + 1) * kD + psi] = om[t][1];
-                    oo[(2 * c) * kD + psi + 1] = om[t][2];
-                    oo[(2 * c + 1) * kD + psi + 1] = om[t][3];
+                    oo[(2 * c) * kHS + swz(psi)] = om[t][0];
+                    oo[(2 * c + 1) * kHS + swz(psi)] = om[t][1];
+                    oo[(2 * c) * kHS + swz(psi + 1)] = om[t][2];
+                    oo[(2 * c + 1) * kHS + swz(psi + 1)] = om[t][3];
                 }
             }
             consumer_sync();
@@ -469,14 +483,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 const int h = idx >> 7, d = idx & (kD - 1);
                 float M = kNegInf;
 #pragma unroll
-                for (int w = 0; w < kDecW; ++w) M = fmaxf(M, scratch[w * kPartFloats + h]);
+                for (int w = 0; w < kDecW; ++w) M = fmaxf(M, scratch[w * kScr + h]);
                 float acc = 0.f, lsum = 0.f;
 #pragma unroll
                 for (int w = 0; w < kDecW; ++w) {
-                    const float mw = scratch[w * kPartFloats + h];
+                    const float mw = scratch[w * kScr + h];
                     const float f = (mw == kNegInf) ? 0.f : exp2f(mw - M);
-                    acc = fmaf(f, scratch[w * kPartFloats + 2 * kMaxG + h * kD + d], acc);
-                    lsum = fmaf(f, scratch[w * kPartFloats + kMaxG + h], lsum);
+                    acc = fmaf(f, scratch[w * kScr + 2 * kMaxG + h * kHS + swz(d)], acc);
+                    lsum = fmaf(f, scratch[w * kScr + kMaxG + h], lsum);
                 }
                 if (whole && p.mode == kModeResident) {
                     float *rp = p.res_part + (int64_t)u * kPartFloats;
