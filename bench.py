@@ -36,15 +36,17 @@ import synth  # noqa: E402
 METRIC = "sparse decode tokens/s/GPU at 128K ctx; % of HBM and PCIe roofline"
 D = 128
 
+# Every workload runs the decode-time append fused into the select launch (nosa_append_select);
+# --unfused launches them separately.
 WORKLOADS = {
     # one layer, batch 1, 16 q / 16 kv heads, 8K context, 32 decode steps, KV in device memory
-    "mha-8k": dict(layers=1, B=1, Hq=16, Hkv=16, L=8192, k_q=16, k_e=48, steps=32, offload=False),
+    "mha-8k": dict(layers=1, B=1, Hq=16, Hkv=16, L=8192, k_q=16, k_e=48, steps=32, offload=False, fuse=True),
     # one layer, batch 8, GQA 16 q / 2 kv heads, 16K context, 128 decode steps, KV in device memory
-    "gqa-16k": dict(layers=1, B=8, Hq=16, Hkv=2, L=16384, k_q=16, k_e=48, steps=128, offload=False),
+    "gqa-16k": dict(layers=1, B=8, Hq=16, Hkv=2, L=16384, k_q=16, k_e=48, steps=128, offload=False, fuse=True),
     # 28-layer stack, batch 32, GQA 16/2, 32K context, 64 decode steps, KV in device memory
-    "stack28-32k": dict(layers=28, B=32, Hq=16, Hkv=2, L=32768, k_q=16, k_e=48, steps=64, offload=False),
+    "stack28-32k": dict(layers=28, B=32, Hq=16, Hkv=2, L=32768, k_q=16, k_e=48, steps=64, offload=False, fuse=True),
     # 28-layer stack, batch 64, GQA 16/2, 128K context, 256 decode steps, KV in pinned host memory
-    "offload28-128k": dict(layers=28, B=64, Hq=16, Hkv=2, L=131072, k_q=16, k_e=48, steps=256, offload=True),
+    "offload28-128k": dict(layers=28, B=64, Hq=16, Hkv=2, L=131072, k_q=16, k_e=48, steps=256, offload=True, fuse=True),
 }
 DEFAULT_WORKLOAD = "offload28-128k"
 
@@ -65,6 +67,8 @@ def describe(c, groups):
         s += ", eviction logits from the fused synthetic eviction head"
     if c.get("split"):
         s += ", decode split: Gamma_e + local attended while select and the cache sync run"
+    if c.get("fuse"):
+        s += ", append and select fused in one launch"
     return s
 
 
@@ -114,6 +118,8 @@ class Workload:
         # the fused eviction head: synthetic weights per layer (e is then computed, not an input)
         self.head = bool(c.get("head", False))
         self.split = bool(c.get("split", False))  # decode Gamma_e + local while select / cache sync run
+        # append and select in one launch (it takes given logits and feeds the one-pass decode)
+        self.fuse = bool(c.get("fuse", False)) and not (self.split or self.head)
         self.W = [tuple(torch.from_numpy(w).to(dev) for w in synth.head_weights(seed, l, self.Hkv))
                   for l in range(self.L)] if self.head else None
         self._prefill(dev)
@@ -211,6 +217,12 @@ class Workload:
             append = ("append", lambda s: lay.append(k, v, e, 1, None, s))
         if self.dense:  # the full-attention comparator: append, then attend to every token
             return [append, ("dense", lambda s: lay.dense_decode(q, out, s))]
+        if self.fuse:
+            calls = [("append_select", lambda s: lay.append_select(k, v, e, q, s))]
+            if self.c["offload"]:
+                calls.append(("cache_sync", lambda s: lay.cache_sync(s)))
+            calls.append(("decode", lambda s: lay.sparse_decode(q, out, s)))
+            return calls
         calls = [append]
         if self.split:
             calls += [("fork", None), ("resident", lambda s: lay.decode_resident(q, s))]
@@ -290,8 +302,9 @@ class Workload:
 
     @property
     def launches_per_step(self):
-        # append, select, [cache plan, cache gather], decode (split: resident + rest)
-        return self.L * self.micro * ((5 if self.c["offload"] else 3) + (1 if self.split else 0))
+        # append, select, [cache plan, cache gather], decode (split: resident + rest; fused: append_select)
+        return self.L * self.micro * ((5 if self.c["offload"] else 3) + (1 if self.split else 0) -
+                                      (1 if self.fuse else 0))
 
 
 # ---------------------------------------------------------------------------------------
@@ -452,8 +465,9 @@ def load_peaks():
 # DRAM bytes per launch from an ncu capture (profiles/dram_traffic.json): used only for the
 # same workload variant and only while the kernel's sources are unchanged since the capture.
 KERNEL_SOURCES = {
-    "select": "nosa_select.cu", "decode": "nosa_decode.cu", "cache_sync": "nosa_cache.cu",
-    "append": "nosa_append.cu",
+    "select": ("nosa_select.cu", "nosa_append_unit.cuh"), "decode": ("nosa_decode.cu",),
+    "cache_sync": ("nosa_cache.cu",), "append": ("nosa_append.cu", "nosa_append_unit.cuh"),
+    "append_select": ("nosa_select.cu", "nosa_append_unit.cuh"),
 }
 
 
@@ -461,19 +475,20 @@ def sources_sha(name):
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_offloadable_b200", "csrc")
-    for f in (KERNEL_SOURCES[name], "nosa_common.cuh", "nosa_internal.cuh"):
+    for f in KERNEL_SOURCES[name] + ("nosa_common.cuh", "nosa_internal.cuh"):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
 
 
-def captured_traffic(name, variant):
+def captured_traffic(name, c, args):
     """(bytes per launch, capture note) for kernel `name` on `variant`, or (None, why not)."""
     try:
         with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
             table = json.load(f)
     except (OSError, ValueError):
         return None, "no capture"
+    variant = traffic_variant(c, args, name)
     for e in table.get("captures", []):
         if e.get("kernel") == name and e.get("variant") == variant:
             if e.get("sources_sha256") != sources_sha(name):
@@ -482,13 +497,15 @@ def captured_traffic(name, variant):
     return None, "no capture of this variant"
 
 
-def traffic_variant(c, args):
-    """The workload variant a traffic capture must match: the workload name plus the options that change
-    the kernels' work (the layer count does not change a launch)."""
+def traffic_variant(c, args, name):
+    """The workload variant a traffic capture of kernel `name` must match: the workload name plus the
+    options that change that kernel's work (the layer count does not change a launch)."""
     v = [args.workload]
     for key in ("ck_bf16", "fill", "head", "split"):
         if c.get(key):
             v.append(key)
+    if name in ("select", "append") and (not c.get("fuse") or c.get("head") or c.get("split")):
+        v.append("unfused")
     return "+".join(v)
 
 
@@ -667,6 +684,7 @@ def run_nosa(args, c, rank, world, dev):
         "decode": U * nsel_mean * (64 * D * 2 * 2 + 64 * 4) + 2 * wl.Bm * c["Hq"] * D * 2,
         "append": U * (2 * D * 2 + 4),
     }
+    algo["append_select"] = algo["select"] + algo["append"]
     n_res = min(c["k_e"], nb_c) + 1  # Gamma_e + the local block
     algo["resident"] = U * n_res * (64 * D * 2 * 2 + 64 * 4) + wl.Bm * c["Hq"] * D * 2
     algo["rest"] = U * max(nsel_mean - n_res, 0) * (64 * D * 2 * 2 + 64 * 4) + 2 * wl.Bm * c["Hq"] * D * 2
@@ -697,11 +715,10 @@ def run_nosa(args, c, rank, world, dev):
     hb = max((k for k in kern if "frac_hbm" in kern[k]), key=lambda k: kern[k]["share"])
     roof_hbm = {"bound": "hbm", "kernel": hb, "achieved": kern[hb]["GBps"], "peak": hbm_peak, "unit": "GB/s",
                 "frac": kern[hb]["frac_hbm"], "traffic": None}
-    variant = traffic_variant(c, args)
     for r in (roof, roof_hbm):
         kname = "cache_sync" if r["kernel"].startswith("cache_sync") else r["kernel"]
         if kname in KERNEL_SOURCES:
-            r["traffic"], r["traffic_source"] = captured_traffic(kname, variant)
+            r["traffic"], r["traffic_source"] = captured_traffic(kname, c, args)
 
     # ---- end to end: host inputs -> device, step, outputs -> host, all inside the timed region ----
     e2e = None
@@ -772,7 +789,7 @@ def run_sweep(args, dev):
     for L in SWEEP["context"]:
         for B in SWEEP["batch"]:
             base = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=16, k_e=48, steps=warmup + steps,
-                        ck_bf16=args.ck_bf16)
+                        ck_bf16=args.ck_bf16, fuse=not args.unfused)
             dense = Workload(dict(base, offload=False), warmup + steps + 1, seed=args.seed, dense=True, device=dev)
             dense_ms, _ = dense.time_steps(warmup, steps)
             del dense
@@ -810,7 +827,7 @@ def run_kq_sweep(args, dev):
                 continue
             for fill in (False, True):
                 c = dict(layers=1, B=64, Hq=16, Hkv=2, L=131072, k_q=kq, k_e=k - kq, offload=True, fill=fill,
-                         ck_bf16=args.ck_bf16)
+                         ck_bf16=args.ck_bf16, fuse=not args.unfused)
                 wl = Workload(c, stat_steps + warmup + steps + 1, seed=args.seed, device=dev, micro=2)
                 prev, gam, miss, nsel = None, [], [], []
                 for t in range(stat_steps):
@@ -867,6 +884,8 @@ def main():
                     help="gamma, misses and throughput against k_q/k, union and fill (one JSON line per point)")
     ap.add_argument("--evict-head", action="store_true",
                     help="compute the eviction logits with the fused synthetic eviction head inside append")
+    ap.add_argument("--unfused", action="store_true",
+                    help="launch the decode-time append and the select separately (default: one launch)")
     ap.add_argument("--split", action="store_true",
                     help="split decode: attend Gamma_e + the local block while select and the cache sync run")
     ap.add_argument("--fill", action="store_true",
@@ -881,6 +900,8 @@ def main():
         c["head"] = True
     if args.split:
         c["split"] = True
+    if args.unfused:
+        c["fuse"] = False
     if args.layers is not None:
         c["layers"] = args.layers
     world = int(os.environ.get("WORLD_SIZE", "1"))

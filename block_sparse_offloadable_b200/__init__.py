@@ -33,7 +33,7 @@ WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC, WS_SPLIT = 0, 1, 2,
 
 # Every extern "C" symbol include/nosa.h declares.
 EXPORTS = ["nosa_validate_config", "nosa_state_bytes", "nosa_workspace_bytes", "nosa_state_init",
-           "nosa_compress_append", "nosa_compress_append_head", "nosa_select", "nosa_cache_sync", "nosa_sparse_decode",
+           "nosa_compress_append", "nosa_compress_append_head", "nosa_select", "nosa_append_select", "nosa_cache_sync", "nosa_sparse_decode",
            "nosa_dense_decode", "nosa_decode_resident", "nosa_decode_rest", "nosa_read_error", "nosa_strerror",
            "nosa_select_noalloc"]
 NOALLOC_SELECT_SCRATCH = 1 << 20
@@ -90,6 +90,7 @@ def lib():
         L.nosa_select.argtypes = [C, S, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_cache_sync.argtypes = [C, S, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_sparse_decode.argtypes = [C, S, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.nosa_append_select.argtypes = [C, S, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_decode_resident.argtypes = [C, S, P, P, ctypes.c_size_t, P, ctypes.c_size_t, P]
         L.nosa_decode_rest.argtypes = [C, S, P, P, P, ctypes.c_size_t, P, P, ctypes.c_size_t, P]
         L.nosa_dense_decode.argtypes = [C, S, P, P, P, ctypes.c_size_t, P]
@@ -185,6 +186,12 @@ def nosa_sparse_decode(cfg, st, q, sel, nsel, block_table, out, ws=None, stream=
 
 def _nbytes(t):
     return 0 if t is None else t.numel() * t.element_size()
+
+
+def nosa_append_select(cfg, st, k_new, v_new, e_new, q, sel, nsel, gq=None, ws=None, stream=None):
+    _check(lib().nosa_append_select(ctypes.byref(cfg), ctypes.byref(st), _ptr(k_new), _ptr(v_new), _ptr(e_new),
+                                    _ptr(q), _ptr(sel), _ptr(nsel), _ptr(gq), _ptr(ws), _nbytes(ws),
+                                    _stream(stream)), "nosa_append_select")
 
 
 def nosa_decode_resident(cfg, st, q, split, ws=None, stream=None):
@@ -288,6 +295,11 @@ class NosaLayer:
 
     def select(self, q, stream=None):
         nosa_select(self.cfg, self.state, q, self.sel, self.nsel, self.gq, self.ws_select, stream)
+
+    def append_select(self, k_new, v_new, e_new, q, stream=None):
+        """The decode append (one token) and the selection in one launch."""
+        nosa_append_select(self.cfg, self.state, k_new, v_new, e_new, q, self.sel, self.nsel, self.gq,
+                           self.ws_select, stream)
 
     def cache_sync(self, stream=None):
         nosa_cache_sync(self.cfg, self.state, self.sel, self.nsel, self.block_table, self.n_fetched, self.ws_cache,

@@ -289,9 +289,10 @@ int nosa_state_init(const nosa_config *c, const nosa_state *st, void *stream) {
 
 namespace {
 // nosa_compress_append with e_new given, or with the eviction head (w1, w2) computing it.
-int append_impl(const nosa_config *c, const nosa_state *st, const uint16_t *k_new, const uint16_t *v_new,
+// Validated parameters of an append (e_new given, or the eviction head w1, w2).
+int make_append(const nosa_config *c, const nosa_state *st, const uint16_t *k_new, const uint16_t *v_new,
                 const float *e_new, const float *w1, const float *w2, int32_t T, const int32_t *lens,
-                void *stream) {
+                AppendParams *out) {
     Geo g;
     int rc;
     if ((rc = nosa_validate_config(c))) return rc;
@@ -326,26 +327,21 @@ int append_impl(const nosa_config *c, const nosa_state *st, const uint16_t *k_ne
     p.offload = c->offload; p.T = T; p.ck_bf16 = (c->flags & NOSA_FLAG_CK_BF16) != 0;
     p.fill = (c->flags & NOSA_FLAG_FILL) != 0;
     p.pool = p.fill ? st->pool : nullptr; p.pool_n = p.fill ? st->pool_n : nullptr;
-    return launch_append(p, static_cast<cudaStream_t>(stream));
-}
-}  // namespace
-
-int nosa_compress_append(const nosa_config *c, const nosa_state *st, const uint16_t *k_new,
-                         const uint16_t *v_new, const float *e_new, int32_t T, const int32_t *lens,
-                         void *stream) {
-    if (!e_new) return NOSA_ERR_ARG;
-    return append_impl(c, st, k_new, v_new, e_new, nullptr, nullptr, T, lens, stream);
+    *out = p;
+    return NOSA_OK;
 }
 
-int nosa_compress_append_head(const nosa_config *c, const nosa_state *st, const uint16_t *k_new,
-                              const uint16_t *v_new, const float *w1, const float *w2, int32_t T,
-                              const int32_t *lens, void *stream) {
-    if (!w1 || !w2) return NOSA_ERR_ARG;
-    return append_impl(c, st, k_new, v_new, nullptr, w1, w2, T, lens, stream);
+int append_impl(const nosa_config *c, const nosa_state *st, const uint16_t *k_new, const uint16_t *v_new,
+                const float *e_new, const float *w1, const float *w2, int32_t T, const int32_t *lens,
+                void *stream) {
+    AppendParams p;
+    const int rc = make_append(c, st, k_new, v_new, e_new, w1, w2, T, lens, &p);
+    return rc ? rc : launch_append(p, static_cast<cudaStream_t>(stream));
 }
 
-int nosa_select(const nosa_config *c, const nosa_state *st, const uint16_t *q, int32_t *sel,
-                int32_t *nsel, int32_t *gq, void *ws, size_t ws_bytes, void *stream) {
+// Validated parameters of a select.
+int make_select(const nosa_config *c, const nosa_state *st, const uint16_t *q, int32_t *sel, int32_t *nsel,
+                int32_t *gq, void *ws, size_t ws_bytes, SelectParams *out) {
     Geo g;
     int rc;
     if ((rc = nosa_validate_config(c))) return rc;
@@ -372,6 +368,43 @@ int nosa_select(const nosa_config *c, const nosa_state *st, const uint16_t *q, i
         p.part_keys = reinterpret_cast<uint64_t *>(static_cast<uint8_t *>(ws) +
                                                    align256((size_t)g.units * sizeof(int32_t)));
     }
+    *out = p;
+    return NOSA_OK;
+}
+}  // namespace
+
+int nosa_compress_append(const nosa_config *c, const nosa_state *st, const uint16_t *k_new,
+                         const uint16_t *v_new, const float *e_new, int32_t T, const int32_t *lens,
+                         void *stream) {
+    if (!e_new) return NOSA_ERR_ARG;
+    return append_impl(c, st, k_new, v_new, e_new, nullptr, nullptr, T, lens, stream);
+}
+
+int nosa_compress_append_head(const nosa_config *c, const nosa_state *st, const uint16_t *k_new,
+                              const uint16_t *v_new, const float *w1, const float *w2, int32_t T,
+                              const int32_t *lens, void *stream) {
+    if (!w1 || !w2) return NOSA_ERR_ARG;
+    return append_impl(c, st, k_new, v_new, nullptr, w1, w2, T, lens, stream);
+}
+
+int nosa_select(const nosa_config *c, const nosa_state *st, const uint16_t *q, int32_t *sel,
+                int32_t *nsel, int32_t *gq, void *ws, size_t ws_bytes, void *stream) {
+    SelectParams p;
+    const int rc = make_select(c, st, q, sel, nsel, gq, ws, ws_bytes, &p);
+    return rc ? rc : launch_select(p, static_cast<cudaStream_t>(stream));
+}
+
+int nosa_append_select(const nosa_config *c, const nosa_state *st, const uint16_t *k_new, const uint16_t *v_new,
+                       const float *e_new, const uint16_t *q, int32_t *sel, int32_t *nsel, int32_t *gq, void *ws,
+                       size_t ws_bytes, void *stream) {
+    if (!e_new) return NOSA_ERR_ARG;
+    AppendParams a;
+    SelectParams p;
+    int rc;
+    if ((rc = make_append(c, st, k_new, v_new, e_new, nullptr, nullptr, 1, nullptr, &a))) return rc;
+    if ((rc = make_select(c, st, q, sel, nsel, gq, ws, ws_bytes, &p))) return rc;
+    p.fused = 1;
+    p.ap = a;
     return launch_select(p, static_cast<cudaStream_t>(stream));
 }
 

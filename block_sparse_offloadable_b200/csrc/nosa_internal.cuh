@@ -50,6 +50,8 @@ struct SelectParams {
     int32_t *pool_n;          // [u]
     int32_t nsub, nblk, G, units, nchunks, chunk_blocks, k_q, k_e, max_sel, ck_bf16, fill;
     float scale;
+    int32_t fused;            // append this step's token first (chunk 0's extra warp), see nosa_select.cu
+    AppendParams ap;          // the append's parameters when fused (T = 1)
 };
 
 struct CacheParams {

@@ -22,7 +22,15 @@
 // (atomic counter, no waiting) merges them into Gamma_q, forms the union with
 // Gamma_e through a block bitmap, appends the local block and writes the
 // ascending selection.
-#include "nosa_internal.cuh"
+//
+// Fused with the decode-time append (nosa_append_select): a sixth warp of each
+// unit's chunk-0 CTA appends the token while the other warps stream.  Nothing
+// the scoring reads changes: the pooled key and the eviction score that the
+// append may complete belong to the local block, which is not a candidate.
+// What does change, Gamma_e (or the fill reading's pool) when a new candidate
+// arrives, is read only by the finalizing CTA, after the counter hand-off, and
+// that CTA writes the new length once every CTA of the unit has read the old.
+#include "nosa_append_unit.cuh"
 
 namespace nosa {
 
@@ -131,7 +139,7 @@ int select_chunk_blocks(int32_t units, int32_t nblk, bool ck_bf16) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectParams p) {
+__global__ void __launch_bounds__((kSelW + 2) * 32) select_kernel(const SelectParams p) {
     constexpr int kSelS = SelGeo<T>::kStages;
     constexpr int kStageBytes = stage_bytes<T>();
     pdl_trigger();  // the successor (cache plan or decode) waits for this grid anyway
@@ -146,7 +154,11 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
 
     const int32_t u = blockIdx.y, chunk = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int32_t L = p.seq_len[u];
+    const int32_t L_prev = p.seq_len[u];
+    const bool grow = p.fused && L_prev >= 0 && L_prev < p.ap.max_ctx;  // this launch appends a token
+    const int32_t L = grow ? L_prev + 1 : L_prev;
+    // a block became a candidate with this token: Gamma_e (or the pool) may change
+    const bool refresh = grow && L_prev >= kBlock && (L_prev & (kBlock - 1)) == 0;
     const int32_t nb_c = L > 0 ? (L - 1) / kBlock : 0;
     const int32_t b0 = min(chunk * p.chunk_blocks, nb_c);
     const int32_t b1 = min(b0 + p.chunk_blocks, nb_c);
@@ -163,7 +175,7 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
 
     // warp 0 may finalize this unit: fetch Gamma_e (fill reading: the head of
     // the pool) now, while the stream runs
-    const int32_t ne = (warp == 0 && !p.fill) ? min(p.gamma_n[u], p.k_e) : 0;
+    int32_t ne = (warp == 0 && !p.fill) ? min(p.gamma_n[u], p.k_e) : 0;
     int32_t pf_n = 0, pf_id = -1;
     if (warp == 0 && p.fill) {
         pf_n = min(max(p.pool_n[u], 0), p.nblk);  // a pool never holds more than nblk - 1 ids
@@ -198,6 +210,12 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
             // never leave with copies in flight
             for (int i = max(0, nstage - kSelS); i < nstage; ++i)
                 if (!mbar_wait(&full[i % kSelS], (i / kSelS) & 1)) set_error(p.err, NOSA_EFLAG_TIMEOUT);
+        }
+    } else if (warp == kSelW + 1) {
+        // the fused append (launched only when fused): chunk 0 of each unit
+        if (chunk == 0) {
+            append_unit(p.ap, u, lane, p.ap.e_new[u], false);
+            __threadfence();  // before the CTA's hand-off to the finalizing CTA
         }
     } else {
         // q_hat = sum of the G query heads of this kv head, lane's 4 dims; the
@@ -272,6 +290,21 @@ __global__ void __launch_bounds__((kSelW + 1) * 32) select_kernel(const SelectPa
             for (int j = 0; j < 8; ++j) list_merge(list, k[j], lane);
         }
     }
+    if (refresh) {  // read again what the fused append may have changed (ordered by the hand-off)
+        if (!p.fill) {
+            ne = min(__ldcg(p.gamma_n + u), p.k_e);
+            const int32_t *ge = p.gamma_e + (int64_t)u * p.k_e;
+#pragma unroll
+            for (int i = 0; i < kMaxKe / 32; ++i) {
+                const int j = lane + 32 * i;
+                ge_reg[i] = (j < ne) ? __ldcg(ge + j) : -1;
+            }
+        } else {
+            pf_n = min(max(__ldcg(p.pool_n + u), 0), p.nblk);
+            pf_id = (lane < pf_n) ? __ldcg(p.pool + (int64_t)u * p.nblk + lane) : -1;
+        }
+    }
+    if (grow && lane == 0) p.ap.seq_len[u] = L;  // every CTA of the unit has read the old length
 
     // ---- finalize: Gamma_q, union with Gamma_e, local block ----
     const int32_t myid = (lane < p.k_q && list != 0ull) ? key_block(list) : -1;
@@ -332,7 +365,8 @@ int launch_select_t(const SelectParams &p, cudaStream_t stream) {
                              (int)smem) != cudaSuccess)
         return NOSA_ERR_CUDA;
     dim3 grid(p.nchunks, p.units);
-    return launch_pdl(select_kernel<T>, grid, dim3((kSelW + 1) * 32), smem, stream, p) == cudaSuccess
+    return launch_pdl(select_kernel<T>, grid, dim3((kSelW + 1 + (p.fused ? 1 : 0)) * 32), smem, stream, p) ==
+                   cudaSuccess
                ? NOSA_OK
                : NOSA_ERR_CUDA;
 }

@@ -262,6 +262,20 @@ int nosa_select(const nosa_config *cfg, const nosa_state *st, const uint16_t *q,
                 int32_t *nsel, int32_t *gq, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * a1 (decode, T = 1) and a2 + a3 in one launch: nosa_compress_append(T = 1)
+ * followed by nosa_select, with the same arguments, results and device errors,
+ * but without a launch between them.  The append runs on an extra warp of
+ * one CTA per unit while the pooled keys stream (the scoring reads nothing the
+ * append writes: the pooled key and eviction score it may complete belong to
+ * the local block, which is never a candidate).  The new Gamma_e (or fill
+ * pool) and length are read and written by the unit's finalizing CTA, after
+ * every CTA of the unit is done.  Eviction logits given (not the fused head).
+ */
+int nosa_append_select(const nosa_config *cfg, const nosa_state *st, const uint16_t *k_new,
+                       const uint16_t *v_new, const float *e_new, const uint16_t *q, int32_t *sel,
+                       int32_t *nsel, int32_t *gq, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * a4 -- block cache synchronisation (offload mode).  NOSA pages: montaan.com
  * "System Optimization (NOSI)" item 2 (block-sized KV units on GPU and CPU;
  * only blocks unused in the current step are swapped out) and item 3 (a

@@ -28,7 +28,7 @@ MAX_ABS, MEAN_ABS, REL_L2 = 1e-2, 1e-3, 1e-2
 
 class Scenario:
     def __init__(self, B, Hq, Hkv, k_q, k_e, L0, steps, offload=False, seed=0, layer=0, lens=None,
-                 max_ctx=None, dense=False, ck_bf16=False, fill=False, head=False, split=False):
+                 max_ctx=None, dense=False, ck_bf16=False, fill=False, head=False, split=False, fused=False):
         self.B, self.Hq, self.Hkv, self.k_q, self.k_e = B, Hq, Hkv, k_q, k_e
         self.G = Hq // Hkv
         self.units = B * Hkv
@@ -41,6 +41,7 @@ class Scenario:
         self.fill = fill
         self.head = head  # eviction logits from the fused head (synthetic weights) instead of inputs
         self.split = split  # decode_resident on a side stream during select / cache_sync, then decode_rest
+        self.fused = fused  # decode steps append and select in one launch (nosa_append_select)
         self.W = synth.head_weights(seed, layer, Hkv) if head else None
 
     def cfg(self):
@@ -109,12 +110,16 @@ def run_gpu(sc, data):
         en = torch.from_numpy(np.ascontiguousarray(E[np.arange(sc.units), idx][:, None])).cuda()
         q = _dev16(Q[t])
         out = torch.empty((sc.B, sc.Hq, 128), dtype=torch.int16, device="cuda")
-        append(kn, vn, en, 1)
+        if sc.fused:
+            lay.append_select(kn, vn, en, q)
+        else:
+            append(kn, vn, en, 1)
         if sc.split:
             cur = torch.cuda.current_stream()
             side.wait_stream(cur)
             lay.decode_resident(q, side)
-        lay.select(q)
+        if not sc.fused:
+            lay.select(q)
         if sc.offload:
             lay.cache_sync()
         if sc.split:

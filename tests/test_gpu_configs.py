@@ -126,6 +126,6 @@ def test_offload28_128k_one_layer_micro_batches():
 @pytest.mark.parametrize("B,L,k,offload", [(256, 131072, 128, False), (32, 32768, 32, True)])
 def test_sweep_corners(B, L, k, offload):
     """Sweep corners: the largest device-resident point (batch 256, 128K, k = 128) and an offload point."""
-    c = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=k // 4, k_e=3 * k // 4, steps=64, offload=offload)
+    c = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=k // 4, k_e=3 * k // 4, steps=64, offload=offload, fuse=True)
     run_config(c, steps=4, micro=2 if offload else 1,
                name=f"sweep B={B} L={L} k={k} {'offload' if offload else 'device'}")
