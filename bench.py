@@ -453,6 +453,20 @@ def aggregate_value(world, batch, steps, ms):
     return world * batch * steps / (ms * 1e-3)
 
 
+def host_cpu():
+    """The host CPU model and its logical core count (the oracle timing runs on one of them)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "logical_cores": os.cpu_count()}
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -572,7 +586,8 @@ def run_reference(args, c, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{args.workload}: " + describe(c, args.host_groups)},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc,
+                             "host": host_cpu()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -653,6 +668,7 @@ def run_nosa(args, c, rank, world, dev):
     # ---- per-kernel durations (events around every launch, eager) + selection stats ----
     events = []
     fetched, nsel_sum, nsel_n = [], 0, 0
+    prev_sel, gammas = None, []
     for _ in range(args.profile_steps):
         feed(step_i)
         # hold the GPU while the host enqueues the whole step, so the events time
@@ -667,6 +683,15 @@ def run_nosa(args, c, rank, world, dev):
         for lay in all_layers:
             nsel_sum += int(lay.nsel.sum())
             nsel_n += lay.units
+        # locality gamma(t) = |Sel(t) & S(t-1)| / |Sel(t)| (Sel(t): S(t) without the local block)
+        cur_sel = [(lay.sel.cpu().numpy(), lay.nsel.cpu().numpy()) for lay in all_layers]
+        if prev_sel is not None:
+            for (s1, n1), (s0, n0) in zip(cur_sel, prev_sel):
+                for u in range(s1.shape[0]):
+                    now = set(s1[u, :n1[u] - 1].tolist())
+                    if now:
+                        gammas.append(len(now & set(s0[u, :n0[u]].tolist())) / len(now))
+        prev_sel = cur_sel
     kt = {}
     for name, l, a, b in events:
         kt.setdefault(name, []).append(a.elapsed_time(b))
@@ -753,7 +778,7 @@ def run_nosa(args, c, rank, world, dev):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         per, count, desc = oracle_sample(c, args.host_groups, args.seed, n_units=4, n_steps=24, budget_s=12.0)
         cv = c["B"] / (per * c["layers"] * c["B"] * c["Hkv"])
-        cpu = {"value": cv, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc}
+        cpu = {"value": cv, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc, "host": host_cpu()}
     if rank != 0:
         return
     line = {
@@ -773,6 +798,9 @@ def run_nosa(args, c, rank, world, dev):
                    "kernel_timing": "select/decode: CUDA graph of all layers replayed; append/cache_sync: events per launch"},
         "roofline": roof, "roofline_hbm": roof_hbm, "kernels": kern, "pcie": pcie_obj,
         "mean_selected_blocks": nsel_mean,
+        "gamma": ({"mean": float(np.mean(gammas)), "min": float(np.min(gammas)),
+                   "floor_k_e_over_k": c["k_e"] / (c["k_q"] + c["k_e"]), "unit_steps": len(gammas)}
+                  if gammas else None),
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
         "clocks": clk, "setup_s": setup_s,
     }
