@@ -51,7 +51,9 @@ __device__ __forceinline__ void gamma_e_worst(const int32_t *ge, int32_t ne, con
 
 // One decode append of unit u by one warp, with the token's eviction logit e_tok.
 // write_len = false leaves seq_len[u] to the caller (the fused append + select
-// writes it once every CTA of the unit has read the old length).
+// writes it once every CTA of the unit has read the old length), and fences the
+// device-side writes before the write-through to host memory, which no one
+// reads before a later kernel and which can be slow while PCIe is busy.
 __device__ __forceinline__ void append_unit(const AppendParams &p, int32_t u, int lane, float e_tok,
                                             bool write_len = true) {
     const int32_t pos = p.seq_len[u];
@@ -100,7 +102,6 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, int32_t u, in
     const uint4 val = reinterpret_cast<const uint4 *>(src)[chunk];
     const int64_t off = (lane < 16 ? 0 : kHalfBlockBytes) + (int64_t)w * kRowBytes + chunk * 16;
     *reinterpret_cast<uint4 *>(dst + off) = val;
-    if (host) *reinterpret_cast<uint4 *>(host + off) = val;  // write-through over PCIe
     if (lane == 0) p.e_store[(int64_t)u * p.max_ctx + pos] = e_tok;
 
     // sub-block complete: its compressed key is the mean of its 16 keys (fp64 sum)
@@ -194,6 +195,8 @@ __device__ __forceinline__ void append_unit(const AppendParams &p, int32_t u, in
         }
     }
     if (write_len && lane == 0) p.seq_len[u] = pos + 1;
+    if (!write_len) __threadfence();  // the fused caller hands off to another CTA next
+    if (host) *reinterpret_cast<uint4 *>(host + off) = val;  // write-through over PCIe, last
 }
 
 }  // namespace nosa

@@ -213,10 +213,7 @@ __global__ void __launch_bounds__((kSelW + 2) * 32) select_kernel(const SelectPa
         }
     } else if (warp == kSelW + 1) {
         // the fused append (launched only when fused): chunk 0 of each unit
-        if (chunk == 0) {
-            append_unit(p.ap, u, lane, p.ap.e_new[u], false);
-            __threadfence();  // before the CTA's hand-off to the finalizing CTA
-        }
+        if (chunk == 0) append_unit(p.ap, u, lane, p.ap.e_new[u], false);  // fences before its hand-off
     } else {
         // q_hat = sum of the G query heads of this kv head, lane's 4 dims; the
         // loads are issued together while the first stages are in flight
