@@ -19,8 +19,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _ROOT = os.path.dirname(_HERE)
 LIB_PATH = os.path.join(_HERE, "_lib", "libnosa.so")
-_SOURCES = ["nosa_api.cu", "nosa_append.cu", "nosa_select.cu", "nosa_cache.cu", "nosa_decode.cu", "nosa_noalloc.cu"]
-_HEADERS = ["nosa_common.cuh", "nosa_internal.cuh"]
+_SOURCES = ["nosa_api.cu", "nosa_append.cu", "nosa_select.cu", "nosa_cache.cu", "nosa_decode.cu", "nosa_noalloc.cu",
+            "nosa_diag.cu"]
+_HEADERS = ["nosa_common.cuh", "nosa_internal.cuh", "nosa_append_unit.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared"]
 
@@ -35,7 +36,7 @@ WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC, WS_SPLIT = 0, 1, 2,
 EXPORTS = ["nosa_validate_config", "nosa_state_bytes", "nosa_workspace_bytes", "nosa_state_init",
            "nosa_compress_append", "nosa_compress_append_head", "nosa_select", "nosa_append_select", "nosa_cache_sync", "nosa_sparse_decode",
            "nosa_dense_decode", "nosa_decode_resident", "nosa_decode_rest", "nosa_read_error", "nosa_strerror",
-           "nosa_select_noalloc"]
+           "nosa_select_noalloc", "nosa_check_wait_timeout"]
 NOALLOC_SELECT_SCRATCH = 1 << 20
 
 
@@ -95,6 +96,7 @@ def lib():
         L.nosa_decode_rest.argtypes = [C, S, P, P, P, ctypes.c_size_t, P, P, ctypes.c_size_t, P]
         L.nosa_dense_decode.argtypes = [C, S, P, P, P, ctypes.c_size_t, P]
         L.nosa_read_error.argtypes = [S, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P]
+        L.nosa_check_wait_timeout.argtypes = [P, ctypes.c_int64, P]
         L.nosa_select_noalloc.argtypes = [C, S, P, P, P, P, P]
         L.nosa_strerror.argtypes = [ctypes.c_int]
         L.nosa_strerror.restype = ctypes.c_char_p
@@ -209,6 +211,11 @@ def nosa_dense_decode(cfg, st, q, out, ws=None, stream=None):
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib().nosa_dense_decode(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(out), _ptr(ws), nbytes,
                                    _stream(stream)), "nosa_dense_decode")
+
+
+def nosa_check_wait_timeout(err, max_cycles, stream=None):
+    """Run the bounded-wait diagnostic into the device word `err` (a 1-element int32 tensor)."""
+    _check(lib().nosa_check_wait_timeout(_ptr(err), int(max_cycles), _stream(stream)), "nosa_check_wait_timeout")
 
 
 def nosa_read_error(st, clear=True, stream=None):

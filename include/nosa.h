@@ -365,6 +365,16 @@ int nosa_decode_rest(const nosa_config *cfg, const nosa_state *st, const uint16_
 int nosa_read_error(const nosa_state *st, uint32_t *flags, int clear, void *stream);
 
 /*
+ * Diagnostic (the pages have no counterpart): runs the library's bounded
+ * mbarrier wait, with a bound of max_cycles SM clock cycles (1 .. 2^32), on a
+ * phase that no thread completes, and sets NOSA_EFLAG_TIMEOUT in the device
+ * word *err when the bound runs out -- the path every pipeline wait of the
+ * library takes if its copies never land.  The kernel then returns normally.
+ *   err  device uint32 [1]
+ */
+int nosa_check_wait_timeout(uint32_t *err, int64_t max_cycles, void *stream);
+
+/*
  * nosa_select without a caller-provided workspace, for callers that cannot
  * allocate device memory (a plug-in that is handed only its inputs and
  * outputs, or a path that must not call cudaMalloc because it may
