@@ -328,8 +328,9 @@ class NosaLayer:
         nosa_dense_decode(self.cfg, self.state, q, out, self.ws_dense, stream)
 
     def decode_step(self, k_new, v_new, e_new, q, out, stream=None):
-        self.append(k_new, v_new, e_new, 1, None, stream)
-        self.select(q, stream)
+        """One decode step of this layer: append + select in one launch, the cache sync (offload),
+        and the sparse decode into `out` (bf16 bits [B][Hq][D])."""
+        self.append_select(k_new, v_new, e_new, q, stream)
         if self.cfg.offload:
             self.cache_sync(stream)
         self.sparse_decode(q, out, stream)
