@@ -64,3 +64,11 @@ def test_unfused_offload28_128k_one_layer_micro_batches():
 def test_unfused_stack28_32k_one_layer():
     c = dict(bench.WORKLOADS["stack28-32k"], fuse=False)
     run_config(c, steps=6, name="stack28-32k layer 0, separate append and select")
+
+
+@pytest.mark.parametrize("offload", [False, True])
+def test_layer_decode_step(offload):
+    """NosaLayer.decode_step, the one-call step the README shows (fused append + select, cache sync,
+    sparse decode)."""
+    _run(H.Scenario(B=2, Hq=16, Hkv=2, k_q=4, k_e=12, L0=64 * 21 + 30, steps=70, offload=offload, seed=15,
+                    layer_step=True))
