@@ -8,7 +8,11 @@
  *   nosa_select           two-stage block scores, Gamma_q, union with Gamma_e and local
  *   nosa_cache_sync       (offload mode) swap blocks: fetch misses host -> device cache
  *   nosa_sparse_decode    exact softmax attention over the selected blocks
- * plus nosa_dense_decode, the full-attention comparator.
+ * or three, with nosa_append_select doing the first two in one launch.  Also:
+ * nosa_compress_append_head (the eviction logits from the fused eviction head),
+ * nosa_decode_resident + nosa_decode_rest (the attention split around the
+ * select and the cache sync), nosa_dense_decode (the full-attention
+ * comparator), nosa_select_noalloc, and the nosa_check_wait_timeout diagnostic.
  *
  * Units.  A "unit" is one (sequence b, kv head g) pair, u = b * heads_kv + g.
  * Blocks are 64 tokens, sub-blocks 16 tokens; block j holds positions
@@ -18,7 +22,8 @@
  *
  * Memory.  The caller allocates every buffer (sizes from nosa_state_bytes and
  * nosa_workspace_bytes).  The library allocates nothing and keeps no state
- * besides a cached driver entry point.  Every call is asynchronous on the
+ * besides a cached driver entry point (and the fixed scratch array of
+ * nosa_select_noalloc).  Every call is asynchronous on the
  * given stream and validates its arguments on the host before launching
  * anything; a non-zero return means nothing was launched.  Conditions only
  * the device can see (a sequence outgrowing max_ctx, a bounded wait running
@@ -109,7 +114,8 @@ typedef struct nosa_config {
  *   ck          fp32 [u][nsub][D]   compressed keys: mean of each 16-token sub-block (device);
  *               bf16 [u][nsub][D] with NOSA_FLAG_CK_BF16
  *   blk_evict   fp64 [u][nblk]      block eviction score E_b, pre-exponential (device)
- *   gamma_e     int32 [u][k_e]      Gamma_e block ids, ascending (device)
+ *   gamma_e     int32 [u][k_e]      Gamma_e block ids, ascending; in E-rank order with
+ *                                   NOSA_FLAG_FILL (device)
  *   gamma_n     int32 [u]           |Gamma_e| (device)
  *   seq_len     int32 [u]           tokens held, L (device)
  *   cache       bf16 [u][nslots][2][64][D]  offload block cache (device; NULL if offload == 0)
