@@ -13,13 +13,18 @@
 //    The sparse decode gives every unit max_sel items (nsel is max_sel or just
 //    below it once the context holds k blocks; the -1 padding past nsel is
 //    skipped), which spares a round of global reads before the first block-id
-//    load; the other work lists count their items with a prefix sum.
+//    load; the other work lists count their items with a prefix sum.  The
+//    work lists: S(t) (sparse decode), every block (dense comparator), and the
+//    split decode's two passes -- Gamma_e + the local block (its softmax state
+//    is kept per unit), then the rest of Gamma_q (merged with that state).
 //  * One producer thread streams the range's blocks (keys + values, plus the
 //    64 eviction logits) into a 6-stage shared-memory ring: four 2-D TMA tile
 //    loads (64 rows x 64 dims, 128-byte swizzle) and one bulk copy per block,
 //    completing on the stage's mbarrier.  The block ids of the next 32 items
 //    are fetched by the whole producer warp at once.
-//  * Four consumer warps each own 16 of a block's 64 tokens.  S^T = K Q^T is
+//  * Two groups of four consumer warps take alternate blocks (stage s always
+//    belongs to group s % 2); in a group each warp owns 16 of a block's 64
+//    tokens.  S^T = K Q^T is
 //    one m16n8k16 bf16 tensor-core tile per 16 dims (M = 16 tokens, N = the
 //    <= 8 query heads of the group, so each K/V byte is read once for all
 //    heads).  Key rows are read straight into A fragments with one 16-byte
@@ -31,16 +36,16 @@
 //    transposed in registers with movmatrix, and O^T += V^T P^T runs as eight
 //    more m16n8k16 tiles whose A fragments are built from 16-byte value loads
 //    with byte permutes (output dims permuted, undone at the store).
-//  * A CTA's range splits into unit segments.  At a segment's end the four
-//    warps merge their (m, l, o) states in shared memory (a padded, swizzled
-//    layout that spreads each warp's fragment-order stores over 32 banks; named
-//    barrier, the
+//  * A CTA's range splits into unit segments.  At a segment's end the eight
+//    warps merge their (m, l, o) states in shared memory (group 0 folded into
+//    group 1, then the four warps, in a padded, swizzled layout that spreads
+//    each warp's fragment-order stores over 32 banks; a named barrier, so the
 //    producer keeps streaming); a segment covering its whole unit writes bf16
 //    output, otherwise the partial state goes to the CTA's workspace slot (only
 //    a CTA's first and last segments can be partial) and the last of the
 //    unit's contributors to finish (atomic counter, no waiting) merges the
 //    partials in CTA order and writes the output.
-//  * The consumers derive segment boundaries from the prefix sums, not from
+//  * The consumers derive segment boundaries from the item offsets, not from
 //    the stream, so all four always meet at the same barriers; a bounded wait
 //    that runs out sets a shared abort flag and the error word, and the rest
 //    of the CTA drains without computing.
