@@ -55,3 +55,19 @@ def test_budget_limits(k_q, k_e):
 def test_all_blocks_fit_in_budget():
     # fewer candidates than k: every block selected, sparse == dense
     _run(H.Scenario(B=2, Hq=8, Hkv=1, k_q=16, k_e=48, L0=64 * 10 + 30, steps=5, seed=8, dense=True))
+
+
+@pytest.mark.parametrize("offload", [False, True])
+def test_units_split_over_several_ctas(offload):
+    # 48 units x 25 selected blocks = 1200 items over 148 decode CTAs: 8 items per CTA, so
+    # every unit is streamed by 4 or 5 CTAs and merged from their partial states; ragged lengths
+    # leave some units below the budget (padded selections).
+    lens = [64 * 30 + 5 + 97 * b for b in range(12)]
+    _run(H.Scenario(B=12, Hq=8, Hkv=4, k_q=8, k_e=16, L0=0, steps=24, offload=offload, seed=21, fused=True,
+                    lens=lens))
+
+
+def test_units_merged_from_many_partials():
+    # 5 units x 289 items (the largest budget, k_q = 32, k_e = 256) over 148 CTAs: each unit is
+    # streamed by about 30 CTAs, and its last contributor merges about 30 partial states.
+    _run(H.Scenario(B=5, Hq=8, Hkv=1, k_q=32, k_e=256, L0=64 * 300 + 33, steps=8, seed=22, fused=True))
