@@ -71,3 +71,11 @@ def test_units_merged_from_many_partials():
     # 5 units x 289 items (the largest budget, k_q = 32, k_e = 256) over 148 CTAs: each unit is
     # streamed by about 30 CTAs, and its last contributor merges about 30 partial states.
     _run(H.Scenario(B=5, Hq=8, Hkv=1, k_q=32, k_e=256, L0=64 * 300 + 33, steps=8, seed=22, fused=True))
+
+
+@pytest.mark.parametrize("Hq,Hkv,offload", [(6, 2, False), (5, 1, True), (12, 2, False), (7, 1, False), (14, 2, True)])
+def test_odd_group_sizes(Hq, Hkv, offload):
+    # G = 3, 5, 6, 7, 7 query heads per kv head: the score sums G heads, the decode tiles carry
+    # G of their 8 head columns, and outputs are strided by G * 128
+    _run(H.Scenario(B=2, Hq=Hq, Hkv=Hkv, k_q=4, k_e=10, L0=64 * 26 + 41, steps=40, offload=offload, seed=30 + Hq,
+                    fused=True))
