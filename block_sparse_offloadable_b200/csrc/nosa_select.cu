@@ -21,7 +21,9 @@
 // per-chunk lists go to the workspace; the last CTA of the unit to finish
 // (atomic counter, no waiting) merges them into Gamma_q, forms the union with
 // Gamma_e through a block bitmap, appends the local block and writes the
-// ascending selection.
+// ascending selection.  List merges (a chain of dependent shuffles each) run as
+// a tree over the consumer warps: first the CTA's four lists, then, in the
+// unit's last CTA, a quarter of the chunk lists per warp.
 //
 // Fused with the decode-time append (nosa_append_select): a sixth warp of each
 // unit's chunk-0 CTA appends the token while the other warps stream.  Nothing
@@ -50,6 +52,11 @@ template <typename T> __host__ __device__ constexpr int stage_bytes() { return k
 // its phases in order (parity waits cannot tell phase p from p + 2).
 static_assert(SelGeo<float>::kStages % kSelW == 0, "each stage must have a single consumer warp");
 static_assert(SelGeo<__nv_bfloat16>::kStages % kSelW == 0, "each stage must have a single consumer warp");
+
+// Named barrier of the kSelW consumer warps (the producer and append warps have left).
+__device__ __forceinline__ void sel_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kSelW * 32) : "memory");
+}
 
 // This lane's 4 dims of one pooled-key row in shared memory.
 __device__ __forceinline__ float4 row4(const uint8_t *tile, int row, int lane, float *) {
@@ -266,29 +273,52 @@ __global__ void __launch_bounds__((kSelW + 2) * 32) select_kernel(const SelectPa
         lists[warp * 32 + lane] = list;
     }
     __syncthreads();
-    if (warp != 0) return;
-    for (int w = 1; w < kSelW; ++w) list_merge(list, lists[w * 32 + lane], lane);
+    if (warp >= kSelW) return;
+    // The consumer warps' lists, then (in the unit's last CTA) the chunk lists, merge as
+    // a tree: a merge is a chain of dependent shuffles, so depth is what costs.
+    // (the first level reads lists 1 and 3 only, so warp 2 may overwrite list 2 at once)
+    if ((warp & 1) == 0) list_merge(list, lists[(warp + 1) * 32 + lane], lane);
+    if (warp == 2) lists[2 * 32 + lane] = list;
+    sel_sync();
+    if (warp == 0) list_merge(list, lists[2 * 32 + lane], lane);
 
     if (p.nchunks > 1) {
-        uint64_t *mine = p.part_keys + ((int64_t)u * p.nchunks + chunk) * 32;
-        mine[lane] = list;
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) s_last = (atomicAdd(&p.counter[u], 1) == p.nchunks - 1);
-        __syncwarp();
+        if (warp == 0) {
+            uint64_t *mine = p.part_keys + ((int64_t)u * p.nchunks + chunk) * 32;
+            mine[lane] = list;
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) s_last = (atomicAdd(&p.counter[u], 1) == p.nchunks - 1);
+        }
+        sel_sync();  // s_last is known to the four warps
         if (!s_last) return;
         __threadfence();
-        if (lane == 0) p.counter[u] = 0;
-        list = 0;
+        if (warp == 0 && lane == 0) p.counter[u] = 0;
+        // warp w folds chunk lists w, w + 4, ...; the loads are issued four at a time
         const uint64_t *all = p.part_keys + (int64_t)u * p.nchunks * 32;
-        for (int c0 = 0; c0 < p.nchunks; c0 += 8) {
-            uint64_t k[8];  // issue the loads together, then merge
+        list = 0;  // a warp without chunks contributes an empty list
+        for (int c0 = warp; c0 < p.nchunks; c0 += 4 * kSelW) {
+            uint64_t k[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) k[j] = (c0 + j < p.nchunks) ? __ldcg(all + (c0 + j) * 32 + lane) : 0ull;
+            for (int j = 0; j < 4; ++j) {
+                const int cj = c0 + j * kSelW;
+                k[j] = cj < p.nchunks ? __ldcg(all + cj * 32 + lane) : 0ull;
+            }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) list_merge(list, k[j], lane);
+            for (int j = 0; j < 4; ++j) {  // conditions uniform over the warp
+                if (c0 + j * kSelW >= p.nchunks) break;
+                if (c0 == warp && j == 0) list = k[0];
+                else list_merge(list, k[j], lane);
+            }
         }
+        lists[warp * 32 + lane] = list;
+        sel_sync();
+        if ((warp & 1) == 0) list_merge(list, lists[(warp + 1) * 32 + lane], lane);
+        if (warp == 2) lists[2 * 32 + lane] = list;
+        sel_sync();
+        if (warp == 0) list_merge(list, lists[2 * 32 + lane], lane);
     }
+    if (warp != 0) return;
     if (refresh) {  // read again what the fused append may have changed (ordered by the hand-off)
         if (!p.fill) {
             ne = min(__ldcg(p.gamma_n + u), p.k_e);
