@@ -115,16 +115,17 @@ constexpr int kMaxUnits = 2048;  // (seq, kv head) units per call: the decode ke
 constexpr int kNumSms = 148;
 
 // Split each unit's `work` items into n chunks (one CTA each) to minimise
-//   ceil(units*n / slots) * (ceil(work/n) + ovh) + merge * n,
-// the wave-quantised time plus the serial merge of the n chunk results by the
-// unit's last CTA; `slots` CTAs run at once, `ovh` is the per-CTA fixed cost and
-// `merge` the cost of merging one chunk's result, both in work items.
+//   ceil(units*n / slots) * (ceil(work/n) + ovh) + merge * (ceil(n/4) + 1),
+// the wave-quantised time plus the merge of the n chunk results by the unit's
+// last CTA, a tree over its four consumer warps (ceil(n/4) + 1 levels); `slots`
+// CTAs run at once, `ovh` is the per-CTA fixed cost and `merge` the cost of one
+// merge level, both in work items.
 inline int best_chunks(int64_t units, int64_t work, int64_t slots, int64_t ovh, int64_t nmax, int64_t merge = 0) {
     if (nmax < 1) nmax = 1;
     int64_t best_n = 1, best_cost = -1;
     for (int64_t n = 1; n <= nmax; ++n) {
         const int64_t waves = (units * n + slots - 1) / slots;
-        const int64_t cost = waves * ((work + n - 1) / n + ovh) + merge * n;
+        const int64_t cost = waves * ((work + n - 1) / n + ovh) + merge * ((n + 3) / 4 + 1);
         if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_n = n; }
     }
     return (int)best_n;

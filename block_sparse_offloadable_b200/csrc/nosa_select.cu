@@ -135,9 +135,10 @@ size_t select_smem_bytes(int32_t nblk) {
 int select_chunk_blocks(int32_t units, int32_t nblk, bool ck_bf16) {
     // candidates per unit are at most nblk - 1; per-CTA fixed cost (pipeline
     // fill, the list merges, the atomic hand-off) ~ the time of 32 fp32 blocks,
-    // i.e. of 64 bf16 blocks; the finalizing CTA's merge of one more chunk list
-    // ~ 2 fp32 blocks (measured: it decides the chunk count only for small
-    // problems, where every split fits in one wave)
+    // i.e. of 64 bf16 blocks; one level of the finalizing CTA's merge tree
+    // (ceil(n/4) + 1 levels for n chunk lists) ~ 2 fp32 blocks (measured: it
+    // decides the chunk count only for small problems, where every split fits
+    // in one wave)
     const int64_t work = nblk > 1 ? nblk - 1 : 1;
     int64_t nmax = (work + kSelSB - 1) / kSelSB;
     if (nmax > kMaxChunks) nmax = kMaxChunks;
