@@ -67,11 +67,49 @@ def test_state_sizes(L):
     assert nosa.nosa_state_bytes(cfg(fill=True), nosa.BUF_POOL_N) == u * 4
 
 
-def test_workspace_sizes_cover_chunks(L):
-    for c in (cfg(), cfg(batch=64, max_ctx=131072 + 256)):
-        for which in (nosa.WS_SELECT, nosa.WS_SPARSE_DECODE, nosa.WS_DENSE_DECODE):
-            n = nosa.nosa_workspace_bytes(c, which)
-            assert n == 0 or n >= 256
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
+def _select_chunks(units, nblk, bf16, sms=148, ctas_per_sm=3, stage_blocks=8, max_chunks=64):
+    # The select launcher's documented chunk model: n chunks per unit minimise the wave-quantised
+    # streaming time plus the depth of the finalizing CTA's merge tree (ceil(n/4) + 1 levels); the
+    # chunk length is then rounded up to whole stages.
+    work = nblk - 1 if nblk > 1 else 1
+    nmax = max(1, min((work + stage_blocks - 1) // stage_blocks, max_chunks))
+    ovh, merge = (64, 4) if bf16 else (32, 2)
+    slots = sms * ctas_per_sm
+    best = min(range(1, nmax + 1),
+               key=lambda n: (((units * n + slots - 1) // slots) * ((work + n - 1) // n + ovh)
+                              + merge * ((n + 3) // 4 + 1), n))
+    per = (work + best - 1) // best
+    per = (per + stage_blocks - 1) // stage_blocks * stage_blocks
+    return max(1, (nblk - 1 + per - 1) // per)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_workspace_sizes_follow_the_launch_geometry(L, bf16):
+    # select: per-unit counters + one 32-key list per chunk; decode: per-unit counters + two partial
+    # states (m[8], l[8], o[8][128] fp32) per decode CTA (one per SM)
+    checked = 0
+    for batch in (1, 8, 32, 64, 256):
+        for heads_kv in (1, 2, 8):
+            for ctx in (4096, 16384, 65536, 131072, 1 << 20):
+                units = batch * heads_kv
+                if units > 2048:
+                    continue
+                c = cfg(batch=batch, heads_q=heads_kv * 2, heads_kv=heads_kv, max_ctx=ctx, ck_bf16=bf16)
+                if nosa.nosa_validate_config(c) != nosa.OK:  # beyond the library's index limits
+                    assert nosa.nosa_workspace_bytes(c, nosa.WS_SELECT) == 0
+                    continue
+                checked += 1
+                n = _select_chunks(units, ctx // 64, bf16)
+                want = _align256(units * 4) + units * n * 32 * 8 if n > 1 else 0
+                assert nosa.nosa_workspace_bytes(c, nosa.WS_SELECT) == want, (batch, heads_kv, ctx, n)
+                dec = _align256(units * 4) + 148 * 2 * (2 * 8 + 8 * 128) * 4
+                assert nosa.nosa_workspace_bytes(c, nosa.WS_SPARSE_DECODE) == dec
+                assert nosa.nosa_workspace_bytes(c, nosa.WS_DENSE_DECODE) == dec
+    assert checked >= 70
 
 
 def test_strerror(L):
