@@ -153,6 +153,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// A 32-bit global load that stays where the program puts it (after the asm statements before it).
+__device__ __forceinline__ int32_t ld_volatile_s32(const int32_t *ptr) {
+    int32_t v;
+    asm volatile("ld.volatile.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
 // Order-preserving map of a finite float onto uint32 (larger float -> larger integer).
 __device__ __forceinline__ uint32_t float_order(float f) {
     uint32_t u = __float_as_uint(f);
@@ -160,7 +167,10 @@ __device__ __forceinline__ uint32_t float_order(float f) {
 }
 
 // Selection key: higher score first, then lower block id.  0 means "no entry".
+// A score of -0.0 is keyed as +0.0: the two are equal scores, so the tie must
+// go to the lower block id (float_order alone would rank -0.0 below +0.0).
 __device__ __forceinline__ uint64_t select_key(float score, int32_t blk) {
+    if (__float_as_uint(score) == 0x80000000u) score = 0.0f;
     return (static_cast<uint64_t>(float_order(score)) << 32) |
            static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(blk));
 }

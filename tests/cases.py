@@ -48,7 +48,9 @@ def build_fixture(spec):
     for pos, val in spec.get("e_spikes", []):
         e[pos] = val
     q = np.zeros((spec["G"], D), np.float32)
-    for h, pairs in enumerate(spec["q"]):
+    for h, val in enumerate(spec.get("q_all", [])):  # head h: every dim = val
+        q[h, :] = val
+    for h, pairs in enumerate(spec.get("q", [])):
         for dim, val in pairs:
             q[h, dim] = val
     Kb = f32_to_bf16_bits_exact(K)

@@ -150,6 +150,17 @@ def run_gpu(sc, data):
     return res
 
 
+def record_stats(name, st):
+    """Append a case's parity statistics (exact / excused-tie counts, boundary ties, errors) as one
+    JSON line to the file named by NOSA_PARITY_STATS, if that variable is set."""
+    import json
+    import os
+    path = os.environ.get("NOSA_PARITY_STATS")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": name, **st}) + "\n")
+
+
 def _tie_ok(sa, sb, smax):
     return abs(sa - sb) <= TIE_REL * max(abs(sa), abs(sb), 1e-6 * smax)
 
@@ -157,7 +168,16 @@ def _tie_ok(sa, sb, smax):
 def new_stats():
     return dict(cmp=0, exact=0, excused=0, diverged=0, unexcused=0, ge_mismatch=0, fetch_cmp=0, fetch_mismatch=0,
                 max_abs=0.0, sum_abs=0.0, n_out=0, max_rel=0.0, dense_max_abs=0.0, dense_max_rel=0.0,
-                gamma_min=1.0)
+                gamma_min=1.0, q_ties=0, e_ties=0)
+
+
+def boundary_ties(scores, k):
+    """1 if the k-th and (k+1)-th largest of `scores` are exactly equal (the tie rule decides
+    which block a top-k takes), else 0."""
+    if k <= 0 or len(scores) <= k:
+        return 0
+    s = np.sort(np.asarray(scores, np.float64))[::-1]
+    return int(s[k - 1] == s[k])
 
 
 def compare_step(st, o, r, q, gsel, ggq, gge, gout, k_q, history_ok, gfetch=None, report=None, tag=None,
@@ -168,6 +188,9 @@ def compare_step(st, o, r, q, gsel, ggq, gge, gout, k_q, history_ok, gfetch=None
     gge: GPU Gamma_e ids (any order) or None; gout: GPU output [G][D] as float.
     Returns the updated history flag (False once the selections have differed)."""
     st["cmp"] += 1
+    st["q_ties"] += boundary_ties(r["scores"], k_q)
+    if gge is not None:
+        st["e_ties"] += boundary_ties(o.E()[: r["nb_c"]], o.k_e)
     gq_set = set(x for x in list(ggq)[:k_q] if x >= 0)
     oq_set = set(r["gq"].tolist())
     ge_set = set(gge.tolist()) if gge is not None else set()

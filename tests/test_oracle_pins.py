@@ -12,7 +12,8 @@ import synth
 from oracle import OracleUnit
 from tests import cases
 
-FIXTURES = ["maxpool_two_stage.json", "gqa_group_sum.json", "tie_lower_index.json", "evict_two_stage.json"]
+FIXTURES = ["maxpool_two_stage.json", "gqa_group_sum.json", "tie_lower_index.json", "evict_two_stage.json",
+            "signed_zero_tie.json"]
 
 
 @pytest.mark.parametrize("name", FIXTURES)
