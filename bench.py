@@ -44,7 +44,9 @@ WORKLOADS = {
     # one layer, batch 8, GQA 16 q / 2 kv heads, 16K context, 128 decode steps, KV in device memory
     "gqa-16k": dict(layers=1, B=8, Hq=16, Hkv=2, L=16384, k_q=16, k_e=48, steps=128, offload=False, fuse=True),
     # 28-layer stack, batch 32, GQA 16/2, 32K context, 64 decode steps, KV in device memory
-    "stack28-32k": dict(layers=28, B=32, Hq=16, Hkv=2, L=32768, k_q=16, k_e=48, steps=64, offload=False, fuse=True),
+    # (its line also carries the library's dense decode on the same inputs)
+    "stack28-32k": dict(layers=28, B=32, Hq=16, Hkv=2, L=32768, k_q=16, k_e=48, steps=64, offload=False, fuse=True,
+                        dense_compare=True),
     # 28-layer stack, batch 64, GQA 16/2, 128K context, 256 decode steps, KV in pinned host memory
     "offload28-128k": dict(layers=28, B=64, Hq=16, Hkv=2, L=131072, k_q=16, k_e=48, steps=256, offload=True, fuse=True),
 }
@@ -94,8 +96,11 @@ class Workload:
     sequence still goes through its layers in order.
     """
 
-    def __init__(self, c, n_steps, seed=0, groups=2, layers=None, device="cuda", micro=1, seq_base=0, dense=False):
+    def __init__(self, c, n_steps, seed=0, groups=2, layers=None, device="cuda", micro=1, seq_base=0, dense=False,
+                 layer0=0):
+        # layer0: index of the first layer built (a test may build one layer deep in the stack)
         self.c, self.seed, self.groups, self.seq_base, self.dense = c, seed, groups, seq_base, dense
+        self.layer0 = layer0
         self.L = layers if layers is not None else c["layers"]
         self.B, self.Hq, self.Hkv = c["B"], c["Hq"], c["Hkv"]
         assert self.B % micro == 0, "batch must split evenly into micro-batches"
@@ -110,24 +115,25 @@ class Workload:
         self.host = {}
         if c["offload"]:
             nbytes = nosa.nosa_state_bytes(self.cfg, nosa.BUF_KV_STORE)
-            for g in range(min(groups, self.L)):
+            for g in sorted({self.kv_layer(l) for l in range(self.L)}):
                 for m in range(micro):
                     self.host[(g, m)] = pinned(nbytes, (g, m))
-        self.layers = [[nosa.NosaLayer(self.cfg, dev, self.host[(l % groups, m)] if self.host else None)
+        self.layers = [[nosa.NosaLayer(self.cfg, dev, self.host[(self.kv_layer(l), m)] if self.host else None)
                         for m in range(micro)] for l in range(self.L)]
         # the fused eviction head: synthetic weights per layer (e is then computed, not an input)
         self.head = bool(c.get("head", False))
         self.split = bool(c.get("split", False))  # decode Gamma_e + local while select / cache sync run
         # append and select in one launch (it takes given logits and feeds the one-pass decode)
         self.fuse = bool(c.get("fuse", False)) and not (self.split or self.head)
-        self.W = [tuple(torch.from_numpy(w).to(dev) for w in synth.head_weights(seed, l, self.Hkv))
+        self.W = [tuple(torch.from_numpy(w).to(dev) for w in synth.head_weights(seed, self.layer0 + l, self.Hkv))
                   for l in range(self.L)] if self.head else None
         self._prefill(dev)
         self._inputs(dev)
 
     def kv_layer(self, l):
-        """Layer index whose synthetic K/V layer l holds (host KV groups alias layers)."""
-        return l % self.groups if self.c["offload"] else l
+        """Layer index whose synthetic K/V the l-th built layer holds (host KV groups alias layers)."""
+        lg = self.layer0 + l
+        return lg % self.groups if self.c["offload"] else lg
 
     def _prefill(self, dev):
         T = self.c["L"]
@@ -143,7 +149,7 @@ class Workload:
                 if self.head:
                     lay.append_head(k, v, self.W[l][0], self.W[l][1], T)
                 else:
-                    synth.e_dev(self.seed, l, self.Bm, self.Hkv, 0, T, e, seq0=s0)
+                    synth.e_dev(self.seed, self.layer0 + l, self.Bm, self.Hkv, 0, T, e, seq0=s0)
                     lay.append(k, v, e, T)
         torch.cuda.synchronize()
         del k, v, e
@@ -169,10 +175,10 @@ class Workload:
                 synth.kv_dev(self.seed, synth.K_STREAM, kl, self.Bm, self.Hkv, L0, n, kk, seq0=s0)
                 synth.kv_dev(self.seed, synth.V_STREAM, kl, self.Bm, self.Hkv, L0, n, vv, seq0=s0)
                 if not self.head:
-                    synth.e_dev(self.seed, l, self.Bm, self.Hkv, L0, n, ee, seq0=s0)
+                    synth.e_dev(self.seed, self.layer0 + l, self.Bm, self.Hkv, L0, n, ee, seq0=s0)
                 base = (l * self.micro + m) * self.part_in
                 for t in range(n):
-                    synth.q_dev(self.seed, l, self.Bm, self.Hq, t, qstate, qt, seq0=s0)
+                    synth.q_dev(self.seed, self.layer0 + l, self.Bm, self.Hq, t, qstate, qt, seq0=s0)
                     row = self.inputs[t]
                     row[base:base + self.q_bytes].view(torch.int16).copy_(qt.view(-1))
                     o = base + self.q_bytes
@@ -313,13 +319,18 @@ L2_BYTES = 126 << 20
 
 
 class L2Flusher:
-    """Writes a buffer twice the size of L2 so the next kernel starts with a cold cache."""
+    """Writes a buffer twice the size of L2, then reads another one, so the next kernel starts with
+    none of its data in L2.  The read leaves L2 holding clean lines: a write alone leaves it full of
+    dirty lines, whose write-back would land inside the timed region as traffic the step never made."""
 
     def __init__(self, dev):
         self.buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        self.buf2 = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
 
     def __call__(self):
         self.buf.fill_(1.0)
+        torch.sum(self.buf2, 0, out=self.sink)
 
 
 def ck_elem(c):
@@ -356,6 +367,8 @@ def time_idempotent(wl, name, reps, flush=None):
                     lay.decode_resident(q)
                 elif name == "rest":
                     lay.decode_rest(q, wl.out_view(l, m))
+                elif name == "dense":
+                    lay.dense_decode(q, wl.out_view(l, m))
                 else:
                     lay.sparse_decode(q, wl.out_view(l, m))
     torch.cuda.synchronize()
@@ -726,9 +739,14 @@ def run_nosa(args, c, rank, world, dev):
         avg = sum(kt["cache_sync"]) / len(kt["cache_sync"])
         gbs = fb * 32768 / (avg * 1e-3) / 1e9
         kern["cache_sync"].update({"bytes": fb * 32768, "GBps": gbs, "frac_pcie": gbs / pcie})
+        step_gbs = sum(fetched) / len(fetched) * 32768 / (ms / args.steps * 1e-3) / 1e9
         pcie_obj = {"fetched_blocks_per_step": sum(fetched) / len(fetched),
                     "fetched_blocks_per_unit_step": fb / U, "achieved_GBps": gbs, "peak_GBps": pcie,
-                    "peak": "measured pinned cudaMemcpyAsync H2D, 1 GiB, this box", "frac": gbs / pcie}
+                    "peak": "measured pinned cudaMemcpyAsync H2D, 1 GiB, this box", "frac": gbs / pcie,
+                    "step_GBps": step_gbs, "step_frac": step_gbs / pcie,
+                    "note": "achieved/frac: the cache sync's own launches, timed one at a time on one stream; "
+                            "step_GBps/step_frac: fetched bytes per step over the device-timed step, in which "
+                            "the micro-batches' fetches overlap the other micro-batch's select and decode"}
     dom = max(kern, key=lambda k: kern[k]["share"])
     if dom == "cache_sync" and pcie_obj:
         roof = {"bound": "pcie", "kernel": "cache_sync (plan + gather)", "achieved": pcie_obj["achieved_GBps"],
@@ -834,7 +852,7 @@ def run_nosa(args, c, rank, world, dev):
         cv = c["B"] / (per * c["layers"] * c["B"] * c["Hkv"])
         cpu = {"value": cv, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc, "host": host_cpu()}
     if rank != 0:
-        return
+        return None
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -858,7 +876,32 @@ def run_nosa(args, c, rank, world, dev):
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
         "clocks": clk, "setup_s": setup_s,
     }
-    print(json.dumps(line), flush=True)
+    return line
+
+
+def run_dense(args, c, rank, world, dev):
+    """The library's dense decode (nosa_dense_decode: every token of the context) on the same
+    configuration and the same seeded inputs as the sparse line, graph-replayed the same way."""
+    n = args.warmup + args.steps + 1
+    wl = Workload(c, n, seed=args.seed, groups=args.host_groups, device=dev, layers=args.layers, micro=1,
+                  seq_base=rank * c["B"], dense=True)
+    ms, _ = wl.time_steps(args.warmup, args.steps)
+    ms = reduce_max_ms(ms, world, dev)
+    small = step_bytes(wl) < 2 * L2_BYTES
+    per = time_idempotent(wl, "dense", reps=3, flush=L2Flusher(dev) if small else None)
+    Lctx = c["L"] + n
+    nbytes = wl.units * ((Lctx + 63) // 64) * (64 * D * 2 * 2 + 64 * 4) + 2 * wl.B * c["Hq"] * D * 2
+    hbm_peak, peak_kind = load_peaks()
+    gbs = nbytes / (per * 1e-3) / 1e9
+    errs = [lay.read_error() for per_layer in wl.layers for lay in per_layer]
+    if any(errs):
+        raise RuntimeError(f"device error flags set in the dense comparator: {errs}")
+    del wl
+    torch.cuda.empty_cache()
+    return {"value": world * c["B"] / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps,
+            "warmup": args.warmup, "path": "append + nosa_dense_decode over all L tokens, every layer",
+            "kernel": {"avg_us": per * 1e3, "bytes": nbytes, "GBps": gbs, "frac_hbm": gbs / hbm_peak,
+                       "peak": f"{peak_kind} (MEASURED_PEAKS.json)"}}
 
 
 SWEEP = dict(batch=(1, 8, 32, 128, 256), context=(32768, 131072), k=(32, 64, 128))
@@ -959,6 +1002,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true",
+                    help="skip the dense-decode comparison of workloads that carry one (stack28-32k)")
     ap.add_argument("--sweep", action="store_true",
                     help="batch x context x k sweep against dense decode (one JSON line per point)")
     ap.add_argument("--ck-bf16", action="store_true", help="store pooled keys as bf16 instead of fp32")
@@ -1006,7 +1051,14 @@ def main():
         run_kq_sweep(args, dev)
         return
     try:
-        run_nosa(args, c, rank, world, dev)
+        line = run_nosa(args, c, rank, world, dev)
+        torch.cuda.empty_cache()
+        if c.get("dense_compare") and not args.no_dense:
+            dense = run_dense(args, c, rank, world, dev)
+            if line is not None:
+                line["dense"] = dict(dense, sparse_speedup=line["value"] / dense["value"])
+        if line is not None:
+            print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -7,8 +7,6 @@ offload configuration), and checks sampled units -- the first and last
 sequence, every kv head -- against the CPU oracle at every step run: selected
 sets (near-ties excused and counted), Gamma_e, outputs, and fetch counts.
 """
-import json
-import os
 
 import numpy as np
 import pytest
@@ -23,20 +21,13 @@ from tests import gpu_harness as H
 pytestmark = pytest.mark.gpu
 
 
-def record(name, st):
-    """Append this workload's parity statistics (exact / excused-tie counts, errors) as one JSON
-    line to the file named by NOSA_PARITY_STATS, if that variable is set."""
-    path = os.environ.get("NOSA_PARITY_STATS")
-    if path:
-        with open(path, "a") as f:
-            f.write(json.dumps({"case": name, **st}) + "\n")
-
-
-def run_config(c, steps, seqs=None, seed=0, micro=1, dense_step=None, name=None):
-    wl = bench.Workload(c, steps, seed=seed, groups=2, layers=1, micro=micro)
+def run_config(c, steps, seqs=None, seed=0, micro=1, dense_step=None, name=None, layer=0, units=None):
+    """Decode `steps` steps of layer `layer` of configuration c as the benchmark launches them;
+    check units (seq, kv head) -- by default every kv head of `seqs` (first and last sequence)."""
+    wl = bench.Workload(c, steps, seed=seed, groups=2, layers=1, micro=micro, layer0=layer)
     G = c["Hq"] // c["Hkv"]
     seqs = seqs if seqs is not None else sorted({0, c["B"] - 1})
-    units = [(b, g) for b in seqs for g in range(c["Hkv"])]
+    units = units if units is not None else [(b, g) for b in seqs for g in range(c["Hkv"])]
     rec = {(b, g): [] for (b, g) in units}
     dense_out = None
     for t in range(steps):
@@ -72,11 +63,11 @@ def run_config(c, steps, seqs=None, seed=0, micro=1, dense_step=None, name=None)
         K = synth.kv_rows(seed, synth.K_STREAM, wl.kv_layer(0), b, g, 0, L0 + steps)
         V = synth.kv_rows(seed, synth.V_STREAM, wl.kv_layer(0), b, g, 0, L0 + steps)
         if c.get("head"):
-            W1, W2 = synth.head_weights(seed, 0, c["Hkv"])
+            W1, W2 = synth.head_weights(seed, layer, c["Hkv"])
             E = oracle.evict_head(V, W1[g], W2[g])
         else:
-            E = synth.e_rows(seed, 0, b, g, 0, L0 + steps)
-        Q = np.stack([synth.q_steps(seed, 0, b, g * G + h, steps)[1] for h in range(G)], axis=1)
+            E = synth.e_rows(seed, layer, b, g, 0, L0 + steps)
+        Q = np.stack([synth.q_steps(seed, layer, b, g * G + h, steps)[1] for h in range(G)], axis=1)
         o = OracleUnit(G=G, k_q=c["k_q"], k_e=c["k_e"], cap=wl.max_ctx, ck_bf16=c.get("ck_bf16", False),
                        fill=c.get("fill", False))
         o.prefill(K[:L0], V[:L0], E[:L0])
@@ -96,7 +87,7 @@ def run_config(c, steps, seqs=None, seed=0, micro=1, dense_step=None, name=None)
         assert v["gamma"] == 0 and v["reselect"] == 0 and v["incremental"] == 0 and v["fetch"] == 0, v
     st["mean_abs"] = st["sum_abs"] / max(st["n_out"], 1)
     assert st["cmp"] == len(units) * steps
-    record(name or str(c), st)
+    H.record_stats(name or str(c), st)
     assert not bad, bad[:3]
     H.assert_parity(st)
     return st
@@ -108,24 +99,36 @@ def test_mha_8k_full():
 
 
 def test_gqa_16k_full():
-    """1 layer, batch 8, GQA 8:1, 16K context, 128 steps: sequences 0 and 7, every step."""
-    run_config(dict(bench.WORKLOADS["gqa-16k"]), steps=128, name="gqa-16k")
+    """1 layer, batch 8, GQA 8:1, 16K context, 128 steps: every sequence and kv head, every step."""
+    run_config(dict(bench.WORKLOADS["gqa-16k"]), steps=128, seqs=list(range(8)), name="gqa-16k")
 
 
-def test_stack28_32k_one_layer():
-    """Batch 32, GQA 8:1, 32K context (one layer of the 28): 8 steps, plus the dense comparator."""
-    run_config(dict(bench.WORKLOADS["stack28-32k"]), steps=8, dense_step=7, name="stack28-32k layer 0")
+@pytest.mark.parametrize("layer", [0, 27])
+def test_stack28_32k_layer(layer):
+    """Batch 32, GQA 8:1, 32K context, layer 0 or 27 of the 28: all 64 decode steps, first and last
+    sequence, both kv heads, plus the dense comparator at the last step."""
+    run_config(dict(bench.WORKLOADS["stack28-32k"]), steps=64, dense_step=63, layer=layer,
+               name=f"stack28-32k layer {layer}")
 
 
-def test_offload28_128k_one_layer_micro_batches():
-    """Batch 64, 128K context, KV in pinned host memory, two micro-batches on two streams."""
-    st = run_config(dict(bench.WORKLOADS["offload28-128k"]), steps=6, micro=2, name="offload28-128k layer 0")
+@pytest.mark.parametrize("layer", [0, 27])
+def test_offload28_128k_layer_micro_batches(layer):
+    """Batch 64, 128K context, KV in pinned host memory (layers 0 and 27 hold the two host KV groups),
+    two micro-batches on two streams: all 256 decode steps, first and last sequence, both kv heads."""
+    st = run_config(dict(bench.WORKLOADS["offload28-128k"]), steps=256, micro=2, layer=layer,
+                    name=f"offload28-128k layer {layer}")
     assert st["fetch_cmp"] > 0
 
 
-@pytest.mark.parametrize("B,L,k,offload", [(256, 131072, 128, False), (32, 32768, 32, True)])
-def test_sweep_corners(B, L, k, offload):
-    """Sweep corners: the largest device-resident point (batch 256, 128K, k = 128) and an offload point."""
+SWEEP_CELLS = sorted({(8, L, k, off) for L in (32768, 131072) for k in (32, 64, 128) for off in (False, True)} |
+                     {(B, 131072, 64, off) for B in (1, 8, 32, 128, 256) for off in (False, True)})
+
+
+@pytest.mark.parametrize("B,L,k,offload", SWEEP_CELLS)
+def test_sweep_cell(B, L, k, offload):
+    """The sweep (1 layer, 16 q / 2 kv heads, k_e = 0.75 k): every (context, k, device / pinned host)
+    cell at batch 8, and every batch at 128K and k = 64, in the launch configuration the sweep times;
+    4 decode steps on two sampled units, the first sequence's kv head 0 and the last one's kv head 1."""
     c = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=k // 4, k_e=3 * k // 4, steps=64, offload=offload, fuse=True)
-    run_config(c, steps=4, micro=2 if offload else 1,
+    run_config(c, steps=4, micro=1, units=[(0, 0), (B - 1, 1)],
                name=f"sweep B={B} L={L} k={k} {'offload' if offload else 'device'}")
