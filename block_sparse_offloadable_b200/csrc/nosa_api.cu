@@ -1,5 +1,6 @@
 // nosa_api.cu -- the C ABI of libnosa: argument validation, buffer sizes,
 // tensor maps and kernel launches.  Declarations and contracts: include/nosa.h.
+#include <algorithm>
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <string.h>
@@ -217,6 +218,11 @@ int run_decode(const nosa_config *c, const nosa_state *st, const uint16_t *q, in
     p.qk_log2 = c->scale * 1.4426950408889634f;
     p.counter = static_cast<int32_t *>(ws);
     p.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + align256((size_t)g.units * sizeof(int32_t)));
+    // S(t) gives every unit max_sel nominal items.  With no more units than decode CTAs, each CTA
+    // streams one equal piece of one unit: a CTA then ends at most one partial state, at its end,
+    // instead of stalling mid-stream on the hand-off of a unit it shares with its neighbour.
+    if (mode == kModeSel && g.units <= decode_ctas())
+        p.pieces = (int32_t)std::min<int64_t>(decode_ctas() / g.units, g.max_sel);
     return launch_decode(p, map, static_cast<cudaStream_t>(stream));
 }
 
@@ -494,3 +500,9 @@ const char *nosa_strerror(int code) {
 }
 
 }  // extern "C"
+
+int nosa::select_args_ok(const nosa_config *c, const nosa_state *st, const uint16_t *q, int32_t *sel, int32_t *nsel,
+                         int32_t *gq, void *ws, size_t ws_bytes) {
+    SelectParams p;
+    return make_select(c, st, q, sel, nsel, gq, ws, ws_bytes, &p);
+}

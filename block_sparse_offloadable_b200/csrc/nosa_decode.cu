@@ -327,10 +327,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     __syncthreads();
     const int64_t W = P[U];
-    // ranges over Ge <= W CTAs, so that every range holds at least one item
+    // Balanced: ranges over Ge <= W CTAs, so that every range holds at least one item.
+    // Pieces: unit c / C, piece c % C (the host keeps C <= every unit's item count).
+    const int32_t C = p.pieces;
     const int32_t Ge = (int32_t)(W < (int64_t)G ? (W > 0 ? W : 1) : (int64_t)G);
-    const int64_t lo = (cta < Ge) ? (int64_t)cta * W / Ge : W;
-    const int64_t hi = (cta < Ge) ? (int64_t)(cta + 1) * W / Ge : W;
+    int64_t lo, hi;
+    if (C > 0) {
+        const int32_t uc = cta / C, rc = cta % C;
+        const int64_t a = uc < U ? P[uc] : W, n = uc < U ? P[uc + 1] - a : 0;
+        lo = a + rc * n / C;
+        hi = a + (rc + 1) * n / C;
+    } else {
+        lo = (cta < Ge) ? (int64_t)cta * W / Ge : W;
+        hi = (cta < Ge) ? (int64_t)(cta + 1) * W / Ge : W;
+    }
     const int32_t n_items = (int32_t)(hi - lo);
 
     if (warp == kConsWarps) {
@@ -518,7 +528,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             if (!whole) {
                 __threadfence();
                 consumer_sync();
-                const int32_t cf = cta_of(P[u], W, Ge), cl = cta_of((int64_t)P[u + 1] - 1, W, Ge);
+                const int32_t cf = C > 0 ? u * C : cta_of(P[u], W, Ge);
+                const int32_t cl = C > 0 ? u * C + C - 1 : cta_of((int64_t)P[u + 1] - 1, W, Ge);
                 if (ctid == 0) s_last = (atomicAdd(&p.counter[u], 1) == cl - cf);
                 consumer_sync();
                 if (s_last) {
@@ -537,7 +548,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                         if (cc > cl) {
                             src[t] = p.res_part + (int64_t)u * kPartFloats;
                         } else {
-                            const int sl = (find_unit(P, U, (int64_t)cc * W / Ge) == u) ? 0 : 1;
+                            const int sl = (C > 0 || find_unit(P, U, (int64_t)cc * W / Ge) == u) ? 0 : 1;
                             src[t] = p.part + (int64_t)(cc * 2 + sl) * kPartFloats;
                         }
                     }
@@ -637,7 +648,8 @@ int launch_decode_t(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t
     if (cudaFuncSetAttribute(decode_kernel<kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return NOSA_ERR_CUDA;
-    return launch_pdl(decode_kernel<kStages>, dim3(decode_ctas()), dim3(kDecThreads), smem, stream, tmap, p) ==
+    const int grid = p.pieces > 0 ? p.units * p.pieces : decode_ctas();
+    return launch_pdl(decode_kernel<kStages>, dim3(grid), dim3(kDecThreads), smem, stream, tmap, p) ==
                    cudaSuccess
                ? NOSA_OK
                : NOSA_ERR_CUDA;

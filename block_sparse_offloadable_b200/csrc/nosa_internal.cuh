@@ -91,6 +91,8 @@ struct DecodeParams {
     int32_t max_sel, G, units;
     float qk_log2;              // scale * log2(e)
     int32_t mode;
+    int32_t pieces;             // 0: balanced ranges over decode_ctas() CTAs; C >= 1: U*C CTAs, CTA c
+                                // streams piece c % C (of C equal pieces) of unit c / C
     const int32_t *gamma_e;     // kModeResident: [u][k_e] ascending, and gamma_n [u]
     const int32_t *gamma_n;
     const int32_t *gq;          // kModeRest: [u][k_q] Gamma_q, -1 padded
@@ -106,6 +108,11 @@ int launch_append(const AppendParams &p, cudaStream_t stream);
 int launch_select(const SelectParams &p, cudaStream_t stream);
 int launch_cache_sync(const CacheParams &p, cudaStream_t stream);
 int launch_decode(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t stream);
+
+// The argument checks of nosa_select (config, state, pointers, workspace), with
+// nothing launched: NOSA_OK or the code nosa_select would return before a launch.
+int select_args_ok(const nosa_config *c, const nosa_state *st, const uint16_t *q, int32_t *sel, int32_t *nsel,
+                   int32_t *gq, void *ws, size_t ws_bytes);
 
 // Launch geometry, shared by the launchers and the workspace-size queries.
 int select_chunk_blocks(int32_t units, int32_t nblk, bool ck_bf16);
