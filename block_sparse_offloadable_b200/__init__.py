@@ -36,7 +36,7 @@ WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC, WS_SPLIT = 0, 1, 2,
 EXPORTS = ["nosa_validate_config", "nosa_state_bytes", "nosa_workspace_bytes", "nosa_state_init",
            "nosa_compress_append", "nosa_compress_append_head", "nosa_select", "nosa_append_select", "nosa_cache_sync", "nosa_sparse_decode",
            "nosa_dense_decode", "nosa_decode_resident", "nosa_decode_rest", "nosa_read_error", "nosa_strerror",
-           "nosa_select_noalloc", "nosa_check_wait_timeout"]
+           "nosa_select_noalloc", "nosa_noalloc_scratch_poison", "nosa_check_wait_timeout"]
 NOALLOC_SELECT_SCRATCH = 1 << 20
 
 
@@ -98,6 +98,7 @@ def lib():
         L.nosa_read_error.argtypes = [S, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, P]
         L.nosa_check_wait_timeout.argtypes = [P, ctypes.c_int64, P]
         L.nosa_select_noalloc.argtypes = [C, S, P, P, P, P, P]
+        L.nosa_noalloc_scratch_poison.argtypes = [ctypes.c_uint8, P]
         L.nosa_strerror.argtypes = [ctypes.c_int]
         L.nosa_strerror.restype = ctypes.c_char_p
         _lib = L
@@ -171,6 +172,11 @@ def nosa_select_noalloc(cfg, st, q, sel, nsel, gq=None, stream=None):
     """nosa_select with its scratch in the library's fixed device array (allocates nothing)."""
     _check(lib().nosa_select_noalloc(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(sel), _ptr(nsel), _ptr(gq),
                                      _stream(stream)), "nosa_select_noalloc")
+
+
+def nosa_noalloc_scratch_poison(byte, stream=None):
+    """Test hook: fill nosa_select_noalloc's shared scratch array with `byte` (stale-contents check)."""
+    _check(lib().nosa_noalloc_scratch_poison(int(byte) & 0xFF, _stream(stream)), "nosa_noalloc_scratch_poison")
 
 
 def nosa_cache_sync(cfg, st, sel, nsel, block_table, n_fetched=None, ws=None, stream=None):

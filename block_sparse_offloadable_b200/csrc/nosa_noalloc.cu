@@ -13,7 +13,8 @@
 // bytes.  Every GPU that loads the library holds it until the process exits.
 // Host code cannot use the array's name as a device address, so the first call
 // on each device resolves the address with cudaGetSymbolAddress (with that
-// device current) and caches it.
+// device current) and caches it.  The stream a call is given must belong to
+// the current device, whose array address is the one passed to the kernel.
 #include <mutex>
 #include <string.h>
 
@@ -55,12 +56,23 @@ extern "C" int nosa_select_noalloc(const nosa_config *cfg, const nosa_state *st,
     const size_t need = nosa_workspace_bytes(cfg, NOSA_WS_SELECT);
     if (need > NOSA_NOALLOC_SELECT_SCRATCH) return NOSA_ERR_CAPACITY;
     void *ws = nullptr;
+    if (need > 0 && (rc = scratch_addr(&ws))) return rc;
+    // every argument check of nosa_select runs before anything is queued on the stream
+    if ((rc = nosa::select_args_ok(cfg, st, q, sel, nsel, gq, ws, need))) return rc;
     if (need > 0) {
-        if ((rc = scratch_addr(&ws))) return rc;
         // the counters must start at zero; the lists are written before they are read
         const size_t counters = (size_t)cfg->batch * cfg->heads_kv * sizeof(int32_t);
         if (cudaMemsetAsync(ws, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
             return NOSA_ERR_CUDA;
     }
     return nosa_select(cfg, st, q, sel, nsel, gq, ws, need, stream);
+}
+
+extern "C" int nosa_noalloc_scratch_poison(uint8_t byte, void *stream) {
+    void *ws = nullptr;
+    const int rc = scratch_addr(&ws);
+    if (rc) return rc;
+    return cudaMemsetAsync(ws, byte, NOSA_NOALLOC_SELECT_SCRATCH, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? NOSA_OK
+               : NOSA_ERR_CUDA;
 }

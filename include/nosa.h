@@ -395,13 +395,26 @@ int nosa_check_wait_timeout(uint32_t *err, int64_t max_cycles, void *stream);
  * function allocates nothing.  Its first call on a device looks up the
  * array's device address (cudaGetSymbolAddress, that device current); make
  * that first call before any stream capture.  Each call clears the array's
- * counters on the stream before the kernel.  All calls on a device share the
- * one array, which keeps the last call's contents: calls that overlap on the
- * GPU (other streams, other threads) race and must not be issued.
+ * counters on the stream before the kernel, after every argument check has
+ * passed: a refused call queues nothing.  `stream` must belong to the current
+ * device: the array's address is looked up for the current device, and the
+ * call does not check the stream's device.  All calls on a device
+ * share the one array, which keeps the last call's contents: calls that
+ * overlap on the GPU (other streams, other threads) race and must not be
+ * issued.
  */
 #define NOSA_NOALLOC_SELECT_SCRATCH (1u << 20)
 int nosa_select_noalloc(const nosa_config *cfg, const nosa_state *st, const uint16_t *q,
                         int32_t *sel, int32_t *nsel, int32_t *gq, void *stream);
+
+/*
+ * Test hook of nosa_select_noalloc (no paper counterpart): fill the whole
+ * shared scratch array of the current device with `byte`, on `stream`, as an
+ * interrupted earlier call could have left it.  A following
+ * nosa_select_noalloc must still give nosa_select's results.  `stream` must
+ * belong to the current device; allocates nothing.
+ */
+int nosa_noalloc_scratch_poison(uint8_t byte, void *stream);
 
 /* Human-readable text of a return code. */
 const char *nosa_strerror(int code);

@@ -33,7 +33,11 @@ def test_noalloc_select_matches_workspace_select(B, Hq, Hkv, k_q, k_e, L0):
                    torch.from_numpy(np.ascontiguousarray(E[idx, L0 + t][:, None])).cuda(), 1)
         q = H._dev16(Q[t])
         lay.select(q)  # the existing entry point, workspace from the caller
-        for _ in range(2):  # two calls in a row on the shared scratch array
+        for rep in range(3):  # two calls in a row on the shared scratch array, then one after a poisoning
+            if rep == 2:
+                # stale counters and lists, as an interrupted call could leave them: the call must
+                # clear what has to start at zero
+                nosa.nosa_noalloc_scratch_poison(0x5A)
             sel2.fill_(-7), nsel2.fill_(-7), gq2.fill_(-7)
             nosa.nosa_select_noalloc(cfg, lay.state, q, sel2, nsel2, gq2)
             torch.cuda.synchronize()
@@ -56,3 +60,47 @@ def test_noalloc_rejects_oversize_workspace():
     with pytest.raises(nosa.NosaError) as ei:
         nosa.nosa_select_noalloc(cfg, st, q, sel, nsel)
     assert ei.value.code == nosa.ERR_CAPACITY
+
+
+def _captured_nodes(fn):
+    """Number of graph nodes that fn() enqueues on a capturing stream (fn's exception is kept)."""
+    import ctypes
+    g = torch.cuda.CUDAGraph(keep_graph=True)  # the raw graph is kept for inspection, never instantiated
+    s = torch.cuda.Stream()
+    raised = None
+    with torch.cuda.stream(s):
+        g.capture_begin(capture_error_mode="thread_local")
+        try:
+            fn(s)
+        except nosa.NosaError as e:
+            raised = e
+        g.capture_end()
+    drv = ctypes.CDLL("libcuda.so.1")
+    n = ctypes.c_size_t(0)
+    assert drv.cuGraphGetNodes(ctypes.c_void_p(g.raw_cuda_graph()), None, ctypes.byref(n)) == 0
+    del g
+    return n.value, raised
+
+
+def test_noalloc_refused_call_queues_nothing():
+    # a missing output pointer is refused with NOSA_ERR_PTR by the checks that precede any work:
+    # the call enqueues no node on the (capturing) stream, in particular no clearing of the shared
+    # counters; a valid call captured the same way enqueues the clear and the kernel
+    sc = H.Scenario(B=4, Hq=16, Hkv=2, k_q=16, k_e=48, L0=64 * 300 + 17, steps=1, seed=32)
+    cfg = sc.cfg()
+    assert nosa.nosa_workspace_bytes(cfg, nosa.WS_SELECT) > 0
+    lay = nosa.NosaLayer(cfg)
+    q = torch.zeros((sc.B, sc.Hq, 128), dtype=torch.int16, device="cuda")
+    nosa.nosa_noalloc_scratch_poison(0x33)  # the array's address is resolved before any capture
+    torch.cuda.synchronize()
+    n_bad, err = _captured_nodes(lambda s: nosa.nosa_select_noalloc(cfg, lay.state, q, None, lay.nsel,
+                                                                      lay.gq, stream=s))
+    assert err is not None and err.code == nosa.ERR_PTR
+    assert n_bad == 0
+    n_ok, err = _captured_nodes(lambda s: nosa.nosa_select_noalloc(cfg, lay.state, q, lay.sel, lay.nsel,
+                                                                     lay.gq, stream=s))
+    assert err is None and n_ok >= 2  # the counter clear and the select kernel
+    # and the next call, run for real on an empty state, leaves no error
+    nosa.nosa_select_noalloc(cfg, lay.state, q, lay.sel, lay.nsel, lay.gq)
+    torch.cuda.synchronize()
+    assert int(lay.nsel.sum()) == 0 and lay.read_error() == 0
