@@ -73,6 +73,8 @@ constexpr float kNegInf = -__builtin_huge_valf();
 // dim XOR-ed with bit 5, so the fragment-order stores of a warp hit 32 distinct banks.
 constexpr int kHS = kD + 1;
 constexpr int kScr = 2 * kMaxG + kMaxG * kHS;
+// Units split into at most this many pieces are merged by their last piece in one pass.
+constexpr int kOnePassPieces = 16;
 __device__ __forceinline__ int swz(int x) { return x ^ ((x >> 5) & 1); }
 
 __device__ __forceinline__ uint32_t word(const uint4 &v, int i) {
@@ -532,7 +534,44 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 const int32_t cl = C > 0 ? u * C + C - 1 : cta_of((int64_t)P[u + 1] - 1, W, Ge);
                 if (ctid == 0) s_last = (atomicAdd(&p.counter[u], 1) == cl - cf);
                 consumer_sync();
-                if (s_last) {
+                if (s_last && C > 0 && C <= kOnePassPieces) {
+                    // last piece of the unit: merge the C pieces' partials (piece order) in one
+                    // pass, every thread loading what its 4 dims need at once
+                    __threadfence();
+                    if (ctid == 0) p.counter[u] = 0;
+                    for (int v = ctid; v < p.G * (kD / 4); v += kConsThreads) {
+                        const int h = v / (kD / 4), d4 = (v % (kD / 4)) * 4;
+                        const float *src0 = p.part + (int64_t)cf * 2 * kPartFloats;  // piece t: slot 0 of CTA cf + t
+                        float mt[kOnePassPieces];
+#pragma unroll
+                        for (int t = 0; t < kOnePassPieces; ++t)
+                            mt[t] = t < C ? __ldcg(src0 + (int64_t)t * 2 * kPartFloats + h) : kNegInf;
+                        float M = kNegInf;
+#pragma unroll
+                        for (int t = 0; t < kOnePassPieces; ++t) M = fmaxf(M, mt[t]);
+                        float ls = 0.f;
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (int t = 0; t < kOnePassPieces; ++t) {
+                            if (t < C) {
+                                const float *st_t = src0 + (int64_t)t * 2 * kPartFloats;
+                                const float f = (mt[t] == kNegInf) ? 0.f : exp2f(mt[t] - M);
+                                const float4 o4 = __ldcg(reinterpret_cast<const float4 *>(st_t + 2 * kMaxG + h * kD + d4));
+                                ls = fmaf(f, __ldcg(st_t + kMaxG + h), ls);
+                                acc.x = fmaf(f, o4.x, acc.x); acc.y = fmaf(f, o4.y, acc.y);
+                                acc.z = fmaf(f, o4.z, acc.z); acc.w = fmaf(f, o4.w, acc.w);
+                            }
+                        }
+                        uint2 pk;
+                        if (ls > 0.f) {
+                            pk.x = pack_bf16x2(acc.x / ls, acc.y / ls);
+                            pk.y = pack_bf16x2(acc.z / ls, acc.w / ls);
+                        } else {
+                            pk.x = pk.y = 0u;
+                        }
+                        *reinterpret_cast<uint2 *>(out + h * kD + d4) = pk;
+                    }
+                } else if (s_last) {
                     // last contributor: merge the unit's partials in CTA order
                     __threadfence();
                     if (ctid == 0) p.counter[u] = 0;

@@ -124,6 +124,22 @@ __device__ __forceinline__ void fill_gamma_e(const SelectParams &p, int32_t u, i
     if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_error(p.err, NOSA_EFLAG_STATE);
 }
 
+// Does this launch append a token to a unit of length L_prev (the fused launch, room left)?
+__device__ __forceinline__ bool appends(const SelectParams &p, int32_t L_prev) {
+    return p.fused && L_prev >= 0 && L_prev < p.ap.max_ctx;
+}
+
+// Candidate blocks [b0, b1) of this chunk, for a unit of length L_prev before this launch's
+// append, and the number of stages that stream them.
+__device__ __forceinline__ int32_t chunk_stages(const SelectParams &p, int32_t chunk, int32_t L_prev, int32_t &b0,
+                                                int32_t &b1) {
+    const int32_t L = appends(p, L_prev) ? L_prev + 1 : L_prev;
+    const int32_t nb_c = L > 0 ? (L - 1) / kBlock : 0;
+    b0 = min(chunk * p.chunk_blocks, nb_c);
+    b1 = min(b0 + p.chunk_blocks, nb_c);
+    return (p.k_q > 0 && b1 > b0) ? (b1 - b0 + kSelSB - 1) / kSelSB : 0;
+}
+
 template <typename T>
 size_t select_smem_bytes(int32_t nblk) {
     constexpr int S = SelGeo<T>::kStages;
@@ -164,15 +180,15 @@ __global__ void __launch_bounds__((kSelW + 2) * 32) select_kernel(const SelectPa
 
     const int32_t u = blockIdx.y, chunk = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int32_t L_prev = p.seq_len[u];
-    const bool grow = p.fused && L_prev >= 0 && L_prev < p.ap.max_ctx;  // this launch appends a token
+    // (the producer reads the length itself, after its first copies are out)
+    const int32_t L_prev = warp == kSelW ? 0 : p.seq_len[u];
+    const bool grow = appends(p, L_prev);  // this launch appends a token
     const int32_t L = grow ? L_prev + 1 : L_prev;
     // a block became a candidate with this token: Gamma_e (or the pool) may change
     const bool refresh = grow && L_prev >= kBlock && (L_prev & (kBlock - 1)) == 0;
     const int32_t nb_c = L > 0 ? (L - 1) / kBlock : 0;
-    const int32_t b0 = min(chunk * p.chunk_blocks, nb_c);
-    const int32_t b1 = min(b0 + p.chunk_blocks, nb_c);
-    const int32_t nstage = (p.k_q > 0 && b1 > b0) ? (b1 - b0 + kSelSB - 1) / kSelSB : 0;
+    int32_t b0, b1;
+    const int32_t nstage = chunk_stages(p, chunk, L_prev, b0, b1);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSelS; ++s) {
@@ -204,21 +220,37 @@ __global__ void __launch_bounds__((kSelW + 2) * 32) select_kernel(const SelectPa
     uint64_t list = 0;
     if (warp == kSelW) {
         if (lane == 0) {
-            for (int i = 0; i < nstage; ++i) {
+            const T *ck = static_cast<const T *>(p.ck) + (int64_t)u * p.nsub * kD;
+            auto issue = [&](int i, int32_t bs, int32_t bend) {
+                const int s = i % kSelS;
+                const uint32_t bytes = (uint32_t)min(kSelSB, bend - bs) * (kSubPerBlock * kD * SelGeo<T>::kElem);
+                mbar_arrive_expect_tx(&full[s], bytes);
+                bulk_load(tiles + s * kStageBytes, ck + (int64_t)bs * kSubPerBlock * kD, bytes, &full[s]);
+            };
+            // The first ring of stages goes out before this thread has the context length: the
+            // chunk is bounded by the largest candidate count max_ctx allows, and the stages of
+            // a longer bound than the real one are only waited for, never consumed.  (Whenever
+            // the chunk has real work, its first block is chunk * chunk_blocks either way.)
+            const int32_t nbc_max = p.nblk - 1;
+            const int32_t b0s = min(chunk * p.chunk_blocks, nbc_max);
+            const int32_t b1s = min(b0s + p.chunk_blocks, nbc_max);
+            const int nspec = (p.k_q > 0 && b1s > b0s) ? min(kSelS, (b1s - b0s + kSelSB - 1) / kSelSB) : 0;
+            for (int i = 0; i < nspec; ++i) issue(i, b0s + i * kSelSB, b1s);
+            // the real bounds (the load follows the copies; the asm above keeps it there)
+            int32_t rb0, rb1;
+            const int32_t nst = chunk_stages(p, chunk, ld_volatile_s32(p.seq_len + u), rb0, rb1);
+            int issued = nspec;
+            for (int i = nspec; i < nst; ++i) {
                 const int s = i % kSelS;
                 if (i >= kSelS && !mbar_wait(&empty[s], ((i / kSelS) - 1) & 1)) {
                     set_error(p.err, NOSA_EFLAG_TIMEOUT);
                     break;
                 }
-                const int32_t bs = b0 + i * kSelSB;
-                const uint32_t bytes = (uint32_t)min(kSelSB, b1 - bs) * (kSubPerBlock * kD * SelGeo<T>::kElem);
-                mbar_arrive_expect_tx(&full[s], bytes);
-                bulk_load(tiles + s * kStageBytes,
-                          static_cast<const T *>(p.ck) + ((int64_t)u * p.nsub + (int64_t)bs * kSubPerBlock) * kD,
-                          bytes, &full[s]);
+                issue(i, rb0 + i * kSelSB, rb1);
+                issued = i + 1;
             }
             // never leave with copies in flight
-            for (int i = max(0, nstage - kSelS); i < nstage; ++i)
+            for (int i = max(0, issued - kSelS); i < issued; ++i)
                 if (!mbar_wait(&full[i % kSelS], (i / kSelS) & 1)) set_error(p.err, NOSA_EFLAG_TIMEOUT);
         }
     } else if (warp == kSelW + 1) {
