@@ -495,7 +495,32 @@ KERNEL_SOURCES = {
     "select": ("nosa_select.cu", "nosa_append_unit.cuh"), "decode": ("nosa_decode.cu",),
     "cache_sync": ("nosa_cache.cu",), "append": ("nosa_append.cu", "nosa_append_unit.cuh"),
     "append_select": ("nosa_select.cu", "nosa_append_unit.cuh"),
+    # kernels that the benchmark's per-kernel pass does not time on its own (prefill, the split
+    # decode's passes, the dense comparator, the cache plan): their captures are checked the same way
+    "dense": ("nosa_decode.cu",), "resident": ("nosa_decode.cu",), "rest": ("nosa_decode.cu",),
+    "cache_plan": ("nosa_cache.cu",), "cache_gather": ("nosa_cache.cu",),
+    "append_head": ("nosa_append.cu", "nosa_append_unit.cuh"),
+    "prefill_store": ("nosa_append.cu", "nosa_append_unit.cuh"),
+    "prefill_pool": ("nosa_append.cu", "nosa_append_unit.cuh"),
+    "prefill_gamma": ("nosa_append.cu", "nosa_append_unit.cuh"),
+    "prefill_head": ("nosa_append.cu", "nosa_append_unit.cuh"),
 }
+
+
+def capture_status():
+    """Every committed ncu capture (profiles/dram_traffic.json) and whether the kernel's sources
+    still match it: 'current', or 'stale' (its counters no longer describe the code)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            table = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    out = {}
+    for e in table.get("captures", []):
+        name = e.get("kernel")
+        ok = name in KERNEL_SOURCES and e.get("sources_sha256") == sources_sha(name)
+        out[f"{name}@{e.get('variant')}"] = "current" if ok else "stale"
+    return out
 
 
 def sources_sha(name):
@@ -873,7 +898,7 @@ def run_nosa(args, c, rank, world, dev):
         "gamma": ({"mean": float(np.mean(gammas)), "min": float(np.min(gammas)),
                    "floor_k_e_over_k": c["k_e"] / (c["k_q"] + c["k_e"]), "unit_steps": len(gammas)}
                   if gammas else None),
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "ncu_captures": capture_status(),
         "clocks": clk, "setup_s": setup_s,
     }
     return line
@@ -1002,6 +1027,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dense-only", action="store_true",
+                    help="run only the library's dense decode on the workload (for profiling it)")
     ap.add_argument("--no-dense", action="store_true",
                     help="skip the dense-decode comparison of workloads that carry one (stack28-32k)")
     ap.add_argument("--sweep", action="store_true",
@@ -1051,6 +1078,11 @@ def main():
         run_kq_sweep(args, dev)
         return
     try:
+        if args.dense_only:  # the dense comparator alone (a profiling target)
+            dense = run_dense(args, c, rank, world, dev)
+            if rank == 0:
+                print(json.dumps({"workload": args.workload, "dense": dense}), flush=True)
+            return
         line = run_nosa(args, c, rank, world, dev)
         torch.cuda.empty_cache()
         if c.get("dense_compare") and not args.no_dense:
