@@ -934,8 +934,10 @@ SWEEP = dict(batch=(1, 8, 32, 128, 256), context=(32768, 131072), k=(32, 64, 128
 
 def run_sweep(args, dev):
     """One JSON line per sweep point: 1 layer, 16 q / 2 kv heads, batch x context x k (k_e = 0.75 k),
-    KV in device memory and in pinned host memory, against dense decode on identical inputs."""
-    steps, warmup = args.steps, args.warmup
+    KV in device memory and in pinned host memory, against dense decode on identical inputs.
+    Every point runs at least 16 warm-up steps: with the largest stores (batch 256 at 128K, 32 GiB)
+    the first ~10 graph-replayed steps after a workload is built run ~0.1 ms slower than the rest."""
+    steps, warmup = args.steps, max(args.warmup, 16)
     for L in SWEEP["context"]:
         for B in SWEEP["batch"]:
             base = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=16, k_e=48, steps=warmup + steps,
