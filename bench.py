@@ -276,9 +276,12 @@ class Workload:
             cur.wait_stream(s)
 
     def time_steps(self, warmup, steps, first=0):
-        """Device ms per step over `steps` graph-replayed steps (L2 flushed per step if it fits in L2)."""
+        """Device ms per step over `steps` graph-replayed steps (L2 flushed per step if it fits in L2).
+        Uses 3 + warmup + steps input steps: 3 eager steps, then `warmup` untimed replays of the captured
+        graph (the first replays of a freshly captured graph can run ~0.1 ms slower at the largest
+        stores), then the timed replays."""
         t = first
-        for _ in range(warmup):
+        for _ in range(3):
             self.cur.copy_(self.inputs[t])
             self.launch_step()
             t += 1
@@ -288,6 +291,11 @@ class Workload:
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
             self.launch_step()
+        torch.cuda.synchronize()
+        for _ in range(warmup):
+            self.cur.copy_(self.inputs[t])
+            t += 1
+            g.replay()
         torch.cuda.synchronize()
         small = step_bytes(self) < 2 * L2_BYTES
         flush = L2Flusher(self.cur.device) if small else None
@@ -907,7 +915,7 @@ def run_nosa(args, c, rank, world, dev):
 def run_dense(args, c, rank, world, dev):
     """The library's dense decode (nosa_dense_decode: every token of the context) on the same
     configuration and the same seeded inputs as the sparse line, graph-replayed the same way."""
-    n = args.warmup + args.steps + 1
+    n = 3 + args.warmup + args.steps + 1
     wl = Workload(c, n, seed=args.seed, groups=args.host_groups, device=dev, layers=args.layers, micro=1,
                   seq_base=rank * c["B"], dense=True)
     ms, _ = wl.time_steps(args.warmup, args.steps)
@@ -935,21 +943,22 @@ SWEEP = dict(batch=(1, 8, 32, 128, 256), context=(32768, 131072), k=(32, 64, 128
 def run_sweep(args, dev):
     """One JSON line per sweep point: 1 layer, 16 q / 2 kv heads, batch x context x k (k_e = 0.75 k),
     KV in device memory and in pinned host memory, against dense decode on identical inputs.
-    Every point runs at least 16 warm-up steps: with the largest stores (batch 256 at 128K, 32 GiB)
-    the first ~10 graph-replayed steps after a workload is built run ~0.1 ms slower than the rest."""
-    steps, warmup = args.steps, max(args.warmup, 16)
+    Every point replays its captured step at least 8 times before timing: with the largest stores
+    (batch 256 at 128K, 32 GiB) the first replays of a freshly captured graph run ~0.1 ms slower."""
+    steps, warmup = args.steps, max(args.warmup, 8)
     for L in SWEEP["context"]:
         for B in SWEEP["batch"]:
-            base = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=16, k_e=48, steps=warmup + steps,
+            base = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=16, k_e=48, steps=3 + warmup + steps,
                         ck_bf16=args.ck_bf16, fuse=not args.unfused)
-            dense = Workload(dict(base, offload=False), warmup + steps + 1, seed=args.seed, dense=True, device=dev)
+            dense = Workload(dict(base, offload=False), 3 + warmup + steps + 1, seed=args.seed, dense=True,
+                             device=dev)
             dense_ms, _ = dense.time_steps(warmup, steps)
             del dense
             torch.cuda.empty_cache()
             for k in SWEEP["k"]:
                 for offload in (False, True):
                     c = dict(base, k_q=k // 4, k_e=3 * k // 4, offload=offload)
-                    wl = Workload(c, warmup + steps + 1, seed=args.seed, device=dev)
+                    wl = Workload(c, 3 + warmup + steps + 1, seed=args.seed, device=dev)
                     ms, _ = wl.time_steps(warmup, steps)
                     errs = [lay.read_error() for per in wl.layers for lay in per]
                     del wl
@@ -980,7 +989,7 @@ def run_kq_sweep(args, dev):
             for fill in (False, True):
                 c = dict(layers=1, B=64, Hq=16, Hkv=2, L=131072, k_q=kq, k_e=k - kq, offload=True, fill=fill,
                          ck_bf16=args.ck_bf16, fuse=not args.unfused)
-                wl = Workload(c, stat_steps + warmup + steps + 1, seed=args.seed, device=dev, micro=2)
+                wl = Workload(c, stat_steps + 3 + warmup + steps + 1, seed=args.seed, device=dev, micro=2)
                 prev, gam, miss, nsel = None, [], [], []
                 for t in range(stat_steps):
                     wl.cur.copy_(wl.inputs[t])
