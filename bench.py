@@ -431,6 +431,16 @@ class ClockSampler:
     def stop(self):
         if self.p is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        # a timed region of a few ms (the one-layer workloads) can end before the first 200 ms sample:
+        # keep sampling until there are a few rows (at most ~1.5 s more)
+        for _ in range(15):
+            try:
+                with open(self.f.name) as fh:
+                    if sum(1 for r in fh if r.strip()) >= 3:
+                        break
+            except OSError:
+                break
+            time.sleep(0.1)
         self.p.terminate()
         self.p.wait()
         self.f.seek(0)

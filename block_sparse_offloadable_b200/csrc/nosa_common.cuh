@@ -160,6 +160,16 @@ __device__ __forceinline__ int32_t ld_volatile_s32(const int32_t *ptr) {
     return v;
 }
 
+// Hand-off counter between CTAs: an atomic add at gpu scope with acquire-release semantics.  Issued
+// by one thread after a barrier of its CTA, it releases every write the CTA made before the barrier
+// to the CTA that later acquires the counter (release is cumulative), and acquires the writes that
+// the earlier arrivals released; a barrier after it extends that to the rest of the CTA.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(void *ctr, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(ctr), "r"(v) : "memory");
+    return old;
+}
+
 // Order-preserving map of a finite float onto uint32 (larger float -> larger integer).
 __device__ __forceinline__ uint32_t float_order(float f) {
     uint32_t u = __float_as_uint(f);

@@ -528,16 +528,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 }
             }
             if (!whole) {
-                __threadfence();
+                // hand-off: the partial is written (barrier), one thread counts it with release
+                // semantics; the unit's last contributor acquired the others' partials with the same
+                // atomic, and the barrier after it orders every thread's loads below after them
                 consumer_sync();
                 const int32_t cf = C > 0 ? u * C : cta_of(P[u], W, Ge);
                 const int32_t cl = C > 0 ? u * C + C - 1 : cta_of((int64_t)P[u + 1] - 1, W, Ge);
-                if (ctid == 0) s_last = (atomicAdd(&p.counter[u], 1) == cl - cf);
+                if (ctid == 0) s_last = ((int32_t)atom_add_acq_rel_gpu(p.counter + u, 1u) == cl - cf);
                 consumer_sync();
                 if (s_last && C > 0 && C <= kOnePassPieces) {
                     // last piece of the unit: merge the C pieces' partials (piece order) in one
                     // pass, every thread loading what its 4 dims need at once
-                    __threadfence();
                     if (ctid == 0) p.counter[u] = 0;
                     for (int v = ctid; v < p.G * (kD / 4); v += kConsThreads) {
                         const int h = v / (kD / 4), d4 = (v % (kD / 4)) * 4;
@@ -573,7 +574,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     }
                 } else if (s_last) {
                     // last contributor: merge the unit's partials in CTA order
-                    __threadfence();
                     if (ctid == 0) p.counter[u] = 0;
                     // the CTA partials (and, merging the rest pass, the resident state)
                     const int nc = cl - cf + 1 + (p.mode == kModeRest ? 1 : 0);  // <= Ge + 1

@@ -319,13 +319,13 @@ __global__ void __launch_bounds__((kSelW + 2) * 32) select_kernel(const SelectPa
         if (warp == 0) {
             uint64_t *mine = p.part_keys + ((int64_t)u * p.nchunks + chunk) * 32;
             mine[lane] = list;
-            __threadfence();
             __syncwarp();
-            if (lane == 0) s_last = (atomicAdd(&p.counter[u], 1) == p.nchunks - 1);
+            // counted with release semantics (the warp's list, and what the CTA wrote before the
+            // block barrier above, e.g. the fused append); the last chunk acquires the others' lists
+            if (lane == 0) s_last = ((int32_t)atom_add_acq_rel_gpu(p.counter + u, 1u) == p.nchunks - 1);
         }
-        sel_sync();  // s_last is known to the four warps
+        sel_sync();  // s_last is known to the four warps, and orders their loads after lane 0's acquire
         if (!s_last) return;
-        __threadfence();
         if (warp == 0 && lane == 0) p.counter[u] = 0;
         // warp w folds chunk lists w, w + 4, ...; the loads are issued four at a time
         const uint64_t *all = p.part_keys + (int64_t)u * p.nchunks * 32;
