@@ -73,8 +73,10 @@ constexpr float kNegInf = -__builtin_huge_valf();
 // dim XOR-ed with bit 5, so the fragment-order stores of a warp hit 32 distinct banks.
 constexpr int kHS = kD + 1;
 constexpr int kScr = 2 * kMaxG + kMaxG * kHS;
-// Units split into at most this many pieces are merged by their last piece in one pass.
+// Units split into at most this many pieces are merged by their last piece in one pass; with at
+// most kFewPieces, all of a thread's loads are issued before any of them is used.
 constexpr int kOnePassPieces = 16;
+constexpr int kFewPieces = 4;
 __device__ __forceinline__ int swz(int x) { return x ^ ((x >> 5) & 1); }
 
 __device__ __forceinline__ uint32_t word(const uint4 &v, int i) {
@@ -544,23 +546,49 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                         const int h = v / (kD / 4), d4 = (v % (kD / 4)) * 4;
                         const float *src0 = p.part + (int64_t)cf * 2 * kPartFloats;  // piece t: slot 0 of CTA cf + t
                         float mt[kOnePassPieces];
-#pragma unroll
-                        for (int t = 0; t < kOnePassPieces; ++t)
-                            mt[t] = t < C ? __ldcg(src0 + (int64_t)t * 2 * kPartFloats + h) : kNegInf;
-                        float M = kNegInf;
-#pragma unroll
-                        for (int t = 0; t < kOnePassPieces; ++t) M = fmaxf(M, mt[t]);
                         float ls = 0.f;
                         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (C <= kFewPieces) {
+                            // few pieces (C = 2 at the configs' sizes): every load at once, one round trip
+                            float lt[kFewPieces];
+                            float4 ot[kFewPieces];
 #pragma unroll
-                        for (int t = 0; t < kOnePassPieces; ++t) {
-                            if (t < C) {
+                            for (int t = 0; t < kFewPieces; ++t) {
                                 const float *st_t = src0 + (int64_t)t * 2 * kPartFloats;
-                                const float f = (mt[t] == kNegInf) ? 0.f : exp2f(mt[t] - M);
-                                const float4 o4 = __ldcg(reinterpret_cast<const float4 *>(st_t + 2 * kMaxG + h * kD + d4));
-                                ls = fmaf(f, __ldcg(st_t + kMaxG + h), ls);
-                                acc.x = fmaf(f, o4.x, acc.x); acc.y = fmaf(f, o4.y, acc.y);
-                                acc.z = fmaf(f, o4.z, acc.z); acc.w = fmaf(f, o4.w, acc.w);
+                                mt[t] = t < C ? __ldcg(st_t + h) : kNegInf;
+                                lt[t] = t < C ? __ldcg(st_t + kMaxG + h) : 0.f;
+                                ot[t] = t < C ? __ldcg(reinterpret_cast<const float4 *>(st_t + 2 * kMaxG + h * kD + d4))
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                            }
+                            float M = kNegInf;
+#pragma unroll
+                            for (int t = 0; t < kFewPieces; ++t) M = fmaxf(M, mt[t]);
+#pragma unroll
+                            for (int t = 0; t < kFewPieces; ++t) {
+                                if (t < C) {
+                                    const float f = (mt[t] == kNegInf) ? 0.f : exp2f(mt[t] - M);
+                                    ls = fmaf(f, lt[t], ls);
+                                    acc.x = fmaf(f, ot[t].x, acc.x); acc.y = fmaf(f, ot[t].y, acc.y);
+                                    acc.z = fmaf(f, ot[t].z, acc.z); acc.w = fmaf(f, ot[t].w, acc.w);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int t = 0; t < kOnePassPieces; ++t)
+                                mt[t] = t < C ? __ldcg(src0 + (int64_t)t * 2 * kPartFloats + h) : kNegInf;
+                            float M = kNegInf;
+#pragma unroll
+                            for (int t = 0; t < kOnePassPieces; ++t) M = fmaxf(M, mt[t]);
+#pragma unroll
+                            for (int t = 0; t < kOnePassPieces; ++t) {
+                                if (t < C) {
+                                    const float *st_t = src0 + (int64_t)t * 2 * kPartFloats;
+                                    const float f = (mt[t] == kNegInf) ? 0.f : exp2f(mt[t] - M);
+                                    const float4 o4 = __ldcg(reinterpret_cast<const float4 *>(st_t + 2 * kMaxG + h * kD + d4));
+                                    ls = fmaf(f, __ldcg(st_t + kMaxG + h), ls);
+                                    acc.x = fmaf(f, o4.x, acc.x); acc.y = fmaf(f, o4.y, acc.y);
+                                    acc.z = fmaf(f, o4.z, acc.z); acc.w = fmaf(f, o4.w, acc.w);
+                                }
                             }
                         }
                         uint2 pk;
