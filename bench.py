@@ -359,8 +359,10 @@ def step_bytes(wl):
 
 
 def time_idempotent(wl, name, reps, flush=None):
-    """Average device time of one launch of an idempotent kernel (select, decode, or the split
-    decode's resident / rest passes): a CUDA graph of that kernel for every layer, replayed back to back."""
+    """Average device time of one launch of a kernel (select, decode, the split decode's resident /
+    rest passes, the dense comparator, or the fused append + select): a CUDA graph of that kernel for
+    every layer, replayed back to back.  All but the fused launch are idempotent; the fused launch
+    appends one token per unit per replay, the same work as in a step, so its replays time it too."""
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -371,6 +373,9 @@ def time_idempotent(wl, name, reps, flush=None):
                 q, _, _, _ = wl.views(wl.cur, l, m)
                 if name == "select":
                     lay.select(q)
+                elif name == "append_select":
+                    _, k, v, e = wl.views(wl.cur, l, m)
+                    lay.append_select(k, v, e, q)
                 elif name == "resident":
                     lay.decode_resident(q)
                 elif name == "rest":
@@ -656,7 +661,7 @@ def run_nosa(args, c, rank, world, dev):
     pcie = measure_pcie_h2d(dev) if c["offload"] else None
     micro = args.micro if args.micro else (2 if c["offload"] else 1)
     # replicas: rank r decodes its own sequences r*B .. (r+1)*B-1 (no exchange between sequences)
-    wl = Workload(c, n_steps, seed=args.seed, groups=args.host_groups, device=dev, layers=args.layers, micro=micro,
+    wl = Workload(c, n_steps + 8, seed=args.seed, groups=args.host_groups, device=dev, layers=args.layers, micro=micro,
                   seq_base=rank * c["B"])
     setup_s = time.time() - t_setup
     stream = torch.cuda.current_stream()
@@ -751,8 +756,10 @@ def run_nosa(args, c, rank, world, dev):
     kt = {}
     for name, l, a, b in events:
         kt.setdefault(name, []).append(a.elapsed_time(b))
-    # select and decode are idempotent: replace their event times by graph-replay times
-    for name in ("select", "decode", "resident", "rest"):
+    # replace the event times (launch included) by graph-replay times: select and decode are
+    # idempotent; each replay of the fused append + select appends one more token (the margin of
+    # the workload's context covers the 4 replays)
+    for name in ("select", "decode", "resident", "rest", "append_select"):
         if name in kt:
             per = time_idempotent(wl, name, reps=3, flush=flush)
             kt[name] = [per] * len(kt[name])
@@ -910,7 +917,8 @@ def run_nosa(args, c, rank, world, dev):
                    "cuda_graph": graph is not None, "micro_batches": wl.micro,
                    "l2": ("L2 flushed (256 MB write) before every timed step; steps timed one by one" if small else
                           f"inputs larger than L2: each step streams {step_bytes(wl) / 1e9:.2f} GB of pooled keys and KV blocks"),
-                   "kernel_timing": "select/decode: CUDA graph of all layers replayed; append/cache_sync: events per launch"},
+                   "kernel_timing": "select, decode, fused append + select: CUDA graph of every layer's launch replayed "
+                                    "(the fused launch appends a token per replay); append, cache_sync: events per launch"},
         "roofline": roof, "roofline_hbm": roof_hbm, "kernels": kern, "pcie": pcie_obj,
         "mean_selected_blocks": nsel_mean,
         "gamma": ({"mean": float(np.mean(gammas)), "min": float(np.min(gammas)),
