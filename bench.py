@@ -125,6 +125,8 @@ class Workload:
         self.split = bool(c.get("split", False))  # decode Gamma_e + local while select / cache sync run
         # append and select in one launch (it takes given logits and feeds the one-pass decode)
         self.fuse = bool(c.get("fuse", False)) and not (self.split or self.head)
+        # the whole step of a layer in one launch (device store, union reading, given logits)
+        self.step = bool(c.get("step", False)) and not (self.split or self.head or c["offload"] or c.get("fill"))
         self.W = [tuple(torch.from_numpy(w).to(dev) for w in synth.head_weights(seed, self.layer0 + l, self.Hkv))
                   for l in range(self.L)] if self.head else None
         self._prefill(dev)
@@ -223,6 +225,8 @@ class Workload:
             append = ("append", lambda s: lay.append(k, v, e, 1, None, s))
         if self.dense:  # the full-attention comparator: append, then attend to every token
             return [append, ("dense", lambda s: lay.dense_decode(q, out, s))]
+        if self.step:
+            return [("step", lambda s: lay.fused_step(k, v, e, q, out, s))]
         if self.fuse:
             calls = [("append_select", lambda s: lay.append_select(k, v, e, q, s))]
             if self.c["offload"]:
@@ -316,7 +320,10 @@ class Workload:
 
     @property
     def launches_per_step(self):
-        # append, select, [cache plan, cache gather], decode (split: resident + rest; fused: append_select)
+        # append, select, [cache plan, cache gather], decode (split: resident + rest; fused: append_select;
+        # fused step: one launch)
+        if self.step:
+            return self.L * self.micro
         return self.L * self.micro * ((5 if self.c["offload"] else 3) + (1 if self.split else 0) -
                                       (1 if self.fuse else 0))
 
@@ -360,9 +367,10 @@ def step_bytes(wl):
 
 def time_idempotent(wl, name, reps, flush=None):
     """Average device time of one launch of a kernel (select, decode, the split decode's resident /
-    rest passes, the dense comparator, or the fused append + select): a CUDA graph of that kernel for
-    every layer, replayed back to back.  All but the fused launch are idempotent; the fused launch
-    appends one token per unit per replay, the same work as in a step, so its replays time it too."""
+    rest passes, the dense comparator, the fused append + select, or the fused step): a CUDA graph of
+    that kernel for every layer, replayed back to back.  All but the fused launches are idempotent;
+    a fused launch appends one token per unit per replay, the same work as in a step, so its replays
+    time it too."""
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -376,6 +384,9 @@ def time_idempotent(wl, name, reps, flush=None):
                 elif name == "append_select":
                     _, k, v, e = wl.views(wl.cur, l, m)
                     lay.append_select(k, v, e, q)
+                elif name == "step":
+                    _, k, v, e = wl.views(wl.cur, l, m)
+                    lay.fused_step(k, v, e, q, wl.out_view(l, m))
                 elif name == "resident":
                     lay.decode_resident(q)
                 elif name == "rest":
@@ -515,12 +526,14 @@ def load_peaks():
 # DRAM bytes per launch from an ncu capture (profiles/dram_traffic.json): used only for the
 # same workload variant and only while the kernel's sources are unchanged since the capture.
 KERNEL_SOURCES = {
-    "select": ("nosa_select.cu", "nosa_append_unit.cuh"), "decode": ("nosa_decode.cu",),
+    "select": ("nosa_select.cu", "nosa_append_unit.cuh"), "decode": ("nosa_decode.cu", "nosa_attend.cuh"),
+    "step": ("nosa_step.cu", "nosa_attend.cuh", "nosa_append_unit.cuh"),
     "cache_sync": ("nosa_cache.cu",), "append": ("nosa_append.cu", "nosa_append_unit.cuh"),
     "append_select": ("nosa_select.cu", "nosa_append_unit.cuh"),
     # kernels that the benchmark's per-kernel pass does not time on its own (prefill, the split
     # decode's passes, the dense comparator, the cache plan): their captures are checked the same way
-    "dense": ("nosa_decode.cu",), "resident": ("nosa_decode.cu",), "rest": ("nosa_decode.cu",),
+    "dense": ("nosa_decode.cu", "nosa_attend.cuh"), "resident": ("nosa_decode.cu", "nosa_attend.cuh"),
+    "rest": ("nosa_decode.cu", "nosa_attend.cuh"),
     "cache_plan": ("nosa_cache.cu",), "cache_gather": ("nosa_cache.cu",),
     "append_head": ("nosa_append.cu", "nosa_append_unit.cuh"),
     "prefill_store": ("nosa_append.cu", "nosa_append_unit.cuh"),
@@ -759,7 +772,7 @@ def run_nosa(args, c, rank, world, dev):
     # replace the event times (launch included) by graph-replay times: select and decode are
     # idempotent; each replay of the fused append + select appends one more token (the margin of
     # the workload's context covers the 4 replays)
-    for name in ("select", "decode", "resident", "rest", "append_select"):
+    for name in ("select", "decode", "resident", "rest", "append_select", "step"):
         if name in kt:
             per = time_idempotent(wl, name, reps=3, flush=flush)
             kt[name] = [per] * len(kt[name])
@@ -773,6 +786,7 @@ def run_nosa(args, c, rank, world, dev):
         "append": U * (2 * D * 2 + 4),
     }
     algo["append_select"] = algo["select"] + algo["append"]
+    algo["step"] = algo["append_select"] + algo["decode"]
     n_res = min(c["k_e"], nb_c) + 1  # Gamma_e + the local block
     algo["resident"] = U * n_res * (64 * D * 2 * 2 + 64 * 4) + wl.Bm * c["Hq"] * D * 2
     algo["rest"] = U * max(nsel_mean - n_res, 0) * (64 * D * 2 * 2 + 64 * 4) + 2 * wl.Bm * c["Hq"] * D * 2
@@ -917,8 +931,9 @@ def run_nosa(args, c, rank, world, dev):
                    "cuda_graph": graph is not None, "micro_batches": wl.micro,
                    "l2": ("L2 flushed (256 MB write) before every timed step; steps timed one by one" if small else
                           f"inputs larger than L2: each step streams {step_bytes(wl) / 1e9:.2f} GB of pooled keys and KV blocks"),
-                   "kernel_timing": "select, decode, fused append + select: CUDA graph of every layer's launch replayed "
-                                    "(the fused launch appends a token per replay); append, cache_sync: events per launch"},
+                   "kernel_timing": "select, decode, fused append + select, fused step: CUDA graph of every layer's "
+                                    "launch replayed (a fused launch appends a token per replay); append, cache_sync: "
+                                    "events per launch"},
         "roofline": roof, "roofline_hbm": roof_hbm, "kernels": kern, "pcie": pcie_obj,
         "mean_selected_blocks": nsel_mean,
         "gamma": ({"mean": float(np.mean(gammas)), "min": float(np.min(gammas)),
@@ -1069,6 +1084,8 @@ def main():
                     help="compute the eviction logits with the fused synthetic eviction head inside append")
     ap.add_argument("--unfused", action="store_true",
                     help="launch the decode-time append and the select separately (default: one launch)")
+    ap.add_argument("--fused-step", action="store_true",
+                    help="device store: the whole step of a layer (append, select, decode) in one launch")
     ap.add_argument("--split", action="store_true",
                     help="split decode: attend Gamma_e + the local block while select and the cache sync run")
     ap.add_argument("--fill", action="store_true",
@@ -1085,6 +1102,8 @@ def main():
         c["split"] = True
     if args.unfused:
         c["fuse"] = False
+    if args.fused_step:
+        c["step"] = True
     if args.layers is not None:
         c["layers"] = args.layers
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -19,9 +19,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _ROOT = os.path.dirname(_HERE)
 LIB_PATH = os.path.join(_HERE, "_lib", "libnosa.so")
-_SOURCES = ["nosa_api.cu", "nosa_append.cu", "nosa_select.cu", "nosa_cache.cu", "nosa_decode.cu", "nosa_noalloc.cu",
-            "nosa_diag.cu"]
-_HEADERS = ["nosa_common.cuh", "nosa_internal.cuh", "nosa_append_unit.cuh"]
+_SOURCES = ["nosa_api.cu", "nosa_append.cu", "nosa_select.cu", "nosa_cache.cu", "nosa_decode.cu", "nosa_step.cu",
+            "nosa_noalloc.cu", "nosa_diag.cu"]
+_HEADERS = ["nosa_common.cuh", "nosa_internal.cuh", "nosa_append_unit.cuh", "nosa_attend.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared"]
 
@@ -30,13 +30,13 @@ EFLAG_CAPACITY, EFLAG_TIMEOUT, EFLAG_NOSLOT, EFLAG_STATE = 1, 2, 4, 8
 FLAG_CK_BF16, FLAG_FILL = 1, 2
 (BUF_KV_STORE, BUF_EVICT_LOGIT, BUF_CK, BUF_BLK_EVICT, BUF_GAMMA_E, BUF_GAMMA_N, BUF_SEQ_LEN, BUF_CACHE,
  BUF_SLOT_BLOCK, BUF_BLOCK_SLOT, BUF_ERR, BUF_POOL, BUF_POOL_N) = range(13)
-WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC, WS_SPLIT = 0, 1, 2, 3, 4
+WS_SELECT, WS_SPARSE_DECODE, WS_DENSE_DECODE, WS_CACHE_SYNC, WS_SPLIT, WS_FUSED_STEP = 0, 1, 2, 3, 4, 5
 
 # Every extern "C" symbol include/nosa.h declares.
 EXPORTS = ["nosa_validate_config", "nosa_state_bytes", "nosa_workspace_bytes", "nosa_state_init",
            "nosa_compress_append", "nosa_compress_append_head", "nosa_select", "nosa_append_select", "nosa_cache_sync", "nosa_sparse_decode",
            "nosa_dense_decode", "nosa_decode_resident", "nosa_decode_rest", "nosa_read_error", "nosa_strerror",
-           "nosa_select_noalloc", "nosa_noalloc_scratch_poison", "nosa_check_wait_timeout"]
+           "nosa_select_noalloc", "nosa_noalloc_scratch_poison", "nosa_check_wait_timeout", "nosa_fused_step"]
 NOALLOC_SELECT_SCRATCH = 1 << 20
 
 
@@ -92,6 +92,7 @@ def lib():
         L.nosa_cache_sync.argtypes = [C, S, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_sparse_decode.argtypes = [C, S, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_append_select.argtypes = [C, S, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.nosa_fused_step.argtypes = [C, S, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.nosa_decode_resident.argtypes = [C, S, P, P, ctypes.c_size_t, P, ctypes.c_size_t, P]
         L.nosa_decode_rest.argtypes = [C, S, P, P, P, ctypes.c_size_t, P, P, ctypes.c_size_t, P]
         L.nosa_dense_decode.argtypes = [C, S, P, P, P, ctypes.c_size_t, P]
@@ -202,6 +203,12 @@ def nosa_append_select(cfg, st, k_new, v_new, e_new, q, sel, nsel, gq=None, ws=N
                                     _stream(stream)), "nosa_append_select")
 
 
+def nosa_fused_step(cfg, st, k_new, v_new, e_new, q, sel, nsel, gq, out, ws=None, stream=None):
+    _check(lib().nosa_fused_step(ctypes.byref(cfg), ctypes.byref(st), _ptr(k_new), _ptr(v_new), _ptr(e_new),
+                                 _ptr(q), _ptr(sel), _ptr(nsel), _ptr(gq), _ptr(out), _ptr(ws), _nbytes(ws),
+                                 _stream(stream)), "nosa_fused_step")
+
+
 def nosa_decode_resident(cfg, st, q, split, ws=None, stream=None):
     _check(lib().nosa_decode_resident(ctypes.byref(cfg), ctypes.byref(st), _ptr(q), _ptr(split), _nbytes(split),
                                       _ptr(ws), _nbytes(ws), _stream(stream)), "nosa_decode_resident")
@@ -296,6 +303,7 @@ class NosaLayer:
         self.ws_dense = None if cfg.offload else ws(WS_DENSE_DECODE)
         self.ws_cache = ws(WS_CACHE_SYNC)
         self.split = None if cfg.flags & FLAG_FILL else ws(WS_SPLIT)
+        self.ws_step = ws(WS_FUSED_STEP)
         nosa_state_init(cfg, self.state)
 
     # one decode step = the four calls, in order
@@ -340,6 +348,12 @@ class NosaLayer:
         if self.cfg.offload:
             self.cache_sync(stream)
         self.sparse_decode(q, out, stream)
+
+    def fused_step(self, k_new, v_new, e_new, q, out, stream=None):
+        """One decode step of this layer in one launch (device store, union reading): append,
+        select and sparse decode into `out` (bf16 bits [B][Hq][D])."""
+        nosa_fused_step(self.cfg, self.state, k_new, v_new, e_new, q, self.sel, self.nsel, self.gq, out,
+                        self.ws_step, stream)
 
     def read_error(self, clear=True, stream=None):
         return nosa_read_error(self.state, clear, stream)

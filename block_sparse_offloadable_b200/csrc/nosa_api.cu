@@ -126,6 +126,24 @@ int select_nchunks(const nosa_config *c, const Geo &g) {
 // Words of the per-unit block bitmap in the split-decode buffer.
 size_t split_bits_words(const Geo &g) { return (size_t)g.nblk / 32 + 1; }
 
+// Workspace of the fused step: [score counter, piece counter, 2 flags] per unit, then each team
+// CTA's top-32 list, each CTA's partial state, and each unit's Gamma_q \ Gamma_e list.
+struct StepWs {
+    int32_t C;
+    size_t keys, parts, rest, total;
+};
+
+StepWs step_ws(const nosa_config *c, const Geo &g) {
+    StepWs w;
+    w.C = step_team_size((int32_t)g.units, (int32_t)g.max_sel);
+    const size_t ctas = (size_t)g.units * w.C;
+    w.keys = align256((size_t)g.units * 4 * sizeof(int32_t));
+    w.parts = w.keys + align256(ctas * 32 * sizeof(uint64_t));
+    w.rest = w.parts + align256(ctas * kPartFloats * sizeof(float));
+    w.total = w.rest + (size_t)g.units * (c->k_q > 0 ? c->k_q : 1) * sizeof(int32_t);
+    return w;
+}
+
 size_t ws_bytes_of(const nosa_config *c, int which) {
     Geo g;
     if (!geo_of(c, &g)) return 0;
@@ -141,6 +159,11 @@ size_t ws_bytes_of(const nosa_config *c, int which) {
     if (which == NOSA_WS_SPLIT)
         return align256((size_t)g.units * kPartFloats * sizeof(float)) +
                (size_t)g.units * split_bits_words(g) * sizeof(uint32_t);
+    if (which == NOSA_WS_FUSED_STEP) {
+        if (c->offload || (c->flags & NOSA_FLAG_FILL)) return 0;
+        const StepWs w = step_ws(c, g);
+        return w.total;
+    }
     return 0;
 }
 
@@ -412,6 +435,64 @@ int nosa_append_select(const nosa_config *c, const nosa_state *st, const uint16_
     p.fused = 1;
     p.ap = a;
     return launch_select(p, static_cast<cudaStream_t>(stream));
+}
+
+int nosa_fused_step(const nosa_config *c, const nosa_state *st, const uint16_t *k_new, const uint16_t *v_new,
+                    const float *e_new, const uint16_t *q, int32_t *sel, int32_t *nsel, int32_t *gq, uint16_t *out,
+                    void *ws, size_t ws_bytes, void *stream) {
+    int rc;
+    if ((rc = nosa_validate_config(c))) return rc;
+    if (c->offload || (c->flags & NOSA_FLAG_FILL)) return NOSA_ERR_UNSUPPORTED;
+    if (!e_new) return NOSA_ERR_ARG;
+    AppendParams a;
+    if ((rc = make_append(c, st, k_new, v_new, e_new, nullptr, nullptr, 1, nullptr, &a))) return rc;
+    if ((rc = check_dev(q, true)) || (rc = check_dev(sel, false)) || (rc = check_dev(nsel, false)) ||
+        (rc = check_dev(out, true)))
+        return rc;
+    if (gq && (rc = check_dev(gq, false))) return rc;
+    if ((rc = check_ws(c, NOSA_WS_FUSED_STEP, ws, ws_bytes))) return rc;
+    Geo g;
+    geo_of(c, &g);
+    CUtensorMap map;
+    if ((rc = kv_tensor_map(&map, a.store, g.units * g.nblk * 2 * kBlock))) return rc;
+    const StepWs w = step_ws(c, g);
+    uint8_t *wb = static_cast<uint8_t *>(ws);
+    StepParams sp;
+    memset(&sp, 0, sizeof(sp));
+    DecodeParams &p = sp.d;
+    p.q = q;
+    p.mode = kModeSel;
+    p.e = st->evict_logit;
+    p.seq_len = st->seq_len;
+    p.out = out;
+    p.err = st->err;
+    p.max_ctx = c->max_ctx;
+    p.blocks_per_unit = (int32_t)g.nblk;
+    p.max_sel = (int32_t)g.max_sel;
+    p.G = (int32_t)g.G;
+    p.units = (int32_t)g.units;
+    p.qk_log2 = c->scale * 1.4426950408889634f;
+    p.pieces = w.C;
+    p.k_e = c->k_e;
+    p.k_q = c->k_q;
+    p.nblk = (int32_t)g.nblk;
+    p.counter = reinterpret_cast<int32_t *>(wb) + g.units;
+    p.part = reinterpret_cast<float *>(wb + w.parts);
+    sp.ap = a;
+    sp.ck = st->ck;
+    sp.gamma_e = st->gamma_e;
+    sp.gamma_n = st->gamma_n;
+    sp.sel = sel;
+    sp.nsel = nsel;
+    sp.gq = c->k_q > 0 ? gq : nullptr;
+    sp.score_ctr = reinterpret_cast<int32_t *>(wb);
+    sp.ready = reinterpret_cast<int32_t *>(wb) + 2 * g.units;
+    sp.part_keys = reinterpret_cast<uint64_t *>(wb + w.keys);
+    sp.rest = reinterpret_cast<int32_t *>(wb + w.rest);
+    sp.nsub = (int32_t)g.nsub;
+    sp.ck_bf16 = (c->flags & NOSA_FLAG_CK_BF16) != 0;
+    sp.scale = c->scale;
+    return launch_step(sp, map, static_cast<cudaStream_t>(stream));
 }
 
 int nosa_cache_sync(const nosa_config *c, const nosa_state *st, const int32_t *sel,

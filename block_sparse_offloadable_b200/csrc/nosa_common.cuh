@@ -170,6 +170,36 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(void *ctr, uint32_t v) 
     return old;
 }
 
+// Flags between CTAs of one grid: a release store that publishes what the storing thread (and,
+// through a barrier or fence before it, its CTA) wrote, and the acquiring load that sees it.
+__device__ __forceinline__ void st_release_gpu(int32_t *flag, int32_t v) {
+    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *flag) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    return v;
+}
+
+// Wait until *flag != 0, acquiring what its writer released; false if the bound (SM clock
+// cycles) ran out.
+__device__ __forceinline__ bool flag_wait(const int32_t *flag, long long limit = kWaitCycles) {
+    if (ld_acquire_gpu(flag)) return true;
+    const long long t0 = clock64();
+    while (!ld_acquire_gpu(flag)) {
+        if (clock64() - t0 > limit) return false;
+        __nanosleep(32);
+    }
+    return true;
+}
+
+// Orders this thread's earlier generic-proxy view of global memory (e.g. data acquired from
+// another CTA) before its later asynchronous-proxy accesses (TMA and bulk copies).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Order-preserving map of a finite float onto uint32 (larger float -> larger integer).
 __device__ __forceinline__ uint32_t float_order(float f) {
     uint32_t u = __float_as_uint(f);
@@ -243,6 +273,32 @@ __device__ __forceinline__ void list_merge(uint64_t &list, uint64_t other, int l
         m = lower ? (m > p ? m : p) : (m < p ? m : p);
     }
     list = m;
+}
+
+// ---- pooled-key scoring -----------------------------------------------------------
+// This lane's 4 dims of one pooled-key row in shared memory (fp32 rows of 512 B, bf16 of 256 B).
+__device__ __forceinline__ float4 row4(const uint8_t *tile, int row, int lane, float *) {
+    return lds128f(tile + row * (kD * 4) + lane * 16);
+}
+__device__ __forceinline__ float4 row4(const uint8_t *tile, int row, int lane, __nv_bfloat16 *) {
+    uint2 w;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(w.x), "=r"(w.y)
+                 : "r"(smem_u32(tile + row * (kD * 2) + lane * 8)));
+    return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+}
+
+// One level of a transpose-reduction of per-lane row values v[0..2N): lanes exchange the half
+// they do not keep (the upper half where lane bit o is set) and add.
+template <int N, int R>
+__device__ __forceinline__ void reduce_level(float (&v)[R], int lane, int o) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const float send = upper ? v[i] : v[i + N];
+        const float keep = upper ? v[i + N] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+    }
 }
 
 // ---- programmatic dependent launch ---------------------------------------------

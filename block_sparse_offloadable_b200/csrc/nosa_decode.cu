@@ -49,14 +49,11 @@
 //    the stream, so all four always meet at the same barriers; a bounded wait
 //    that runs out sets a shared abort flag and the error word, and the rest
 //    of the CTA drains without computing.
-#include "nosa_internal.cuh"
+#include "nosa_attend.cuh"
 
 namespace nosa {
 
 namespace {
-constexpr int kDecW = 4;                  // warps per consumer group (16 tokens of a block each)
-constexpr int kGroups = 2;                // consumer groups, taking alternate blocks
-constexpr int kConsWarps = kDecW * kGroups;
 // Ring stages (one block each; one CTA per SM).  The resident pass of the
 // split decode uses fewer, so that one of its CTAs and one select CTA fit on an
 // SM together and the two kernels really run concurrently.
@@ -64,29 +61,6 @@ constexpr int kDecS = 6;
 constexpr int kDecSResident = 4;
 static_assert(kDecS % kGroups == 0 && kDecSResident % kGroups == 0,
               "stage s must always be consumed by group s % kGroups");
-constexpr int kBoxBytes = 64 * 128;       // one TMA box: 64 rows x 64 bf16
-constexpr int kDecThreads = (kConsWarps + 1) * 32;
-constexpr int kConsThreads = kConsWarps * 32;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kNegInf = -__builtin_huge_valf();
-// Merge scratch per warp: m[8], l[8], o[8][kHS] with a padded head row and bit 0 of the
-// dim XOR-ed with bit 5, so the fragment-order stores of a warp hit 32 distinct banks.
-constexpr int kHS = kD + 1;
-constexpr int kScr = 2 * kMaxG + kMaxG * kHS;
-// Units split into at most this many pieces are merged by their last piece in one pass; with at
-// most kFewPieces, all of a thread's loads are issued before any of them is used.
-constexpr int kOnePassPieces = 16;
-constexpr int kFewPieces = 4;
-__device__ __forceinline__ int swz(int x) { return x ^ ((x >> 5) & 1); }
-
-__device__ __forceinline__ uint32_t word(const uint4 &v, int i) {
-    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
-}
-
-__device__ __forceinline__ void consumer_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsThreads) : "memory");
-}
-
 // Work items of unit u in the kernel's mode.
 __device__ __forceinline__ int32_t unit_work(const DecodeParams &p, int32_t u) {
     const int32_t L = p.seq_len[u];
@@ -152,113 +126,6 @@ __device__ __forceinline__ int32_t cta_of(int64_t x, int64_t W, int32_t G) {
     return (int32_t)(((x + 1) * G - 1) / W);
 }
 
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                              uint32_t *err) {
-    if (*abort_flag) return false;
-    if (mbar_wait(bar, parity)) return true;
-    *abort_flag = 1;
-    set_error(err, NOSA_EFLAG_TIMEOUT);
-    return false;
-}
-
-// Per-lane online-softmax state of one consumer warp (heads 2c, 2c+1 of the group).
-struct WarpState {
-    float o[8][4];
-    float m0, m1, l0, l1;
-    __device__ __forceinline__ void reset() {
-#pragma unroll
-        for (int t = 0; t < 8; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
-        m0 = m1 = kNegInf;
-        l0 = l1 = 0.f;
-    }
-};
-
-// Attention of this warp's 16 tokens of one staged block.
-__device__ __forceinline__ void attend_block(WarpState &st, const uint32_t (&qf)[8][2], const uint8_t *t,
-                                             const float *eb, int32_t lb, int32_t L, float qk_log2,
-                                             int warp, int c, int sig) {
-    const int rowA = warp * 16 + sig, rowB = rowA + 8;   // key rows of C rows r, r+8
-    const int vt0 = warp * 16 + c;                        // value rows of k = 2c, 2c+1, 2c+8, 2c+9
-    const int off0 = ((sig ^ c) << 4), off1 = ((sig ^ (c + 4)) << 4);
-    // ---- S^T (16 tokens x 8 heads) = K Q^T, two independent accumulation chains ----
-    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-    float sacc2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint8_t *box = t + (j >> 1) * kBoxBytes;
-        const int sw = (((j & 1) << 2) + c) ^ sig;
-        const uint4 ka = lds128(box + rowA * 128 + (sw << 4));
-        const uint4 kb = lds128(box + rowB * 128 + (sw << 4));
-        const uint32_t a0[4] = {ka.x, kb.x, ka.y, kb.y};
-        const uint32_t a1[4] = {ka.z, kb.z, ka.w, kb.w};
-        mma_16816(sacc, a0, qf[2 * j]);
-        mma_16816(sacc2, a1, qf[2 * j + 1]);
-    }
-#pragma unroll
-    for (int x = 0; x < 4; ++x) sacc[x] += sacc2[x];
-    // ---- online softmax over the 16 tokens, per head (2c, 2c+1) ----
-    const int64_t posA = (int64_t)lb * kBlock + rowA, posB = posA + 8;
-    const float eA = eb[rowA] * kLog2e, eB = eb[rowB] * kLog2e;
-    const float x0 = posA < L ? fmaf(sacc[0], qk_log2, eA) : kNegInf;
-    const float x1 = posA < L ? fmaf(sacc[1], qk_log2, eA) : kNegInf;
-    const float x2 = posB < L ? fmaf(sacc[2], qk_log2, eB) : kNegInf;
-    const float x3 = posB < L ? fmaf(sacc[3], qk_log2, eB) : kNegInf;
-    float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
-#pragma unroll
-    for (int sh = 4; sh < 32; sh <<= 1) {
-        bm0 = fmaxf(bm0, __shfl_xor_sync(0xFFFFFFFFu, bm0, sh));
-        bm1 = fmaxf(bm1, __shfl_xor_sync(0xFFFFFFFFu, bm1, sh));
-    }
-    const float mn0 = fmaxf(st.m0, bm0), mn1 = fmaxf(st.m1, bm1);
-    const float c0 = (mn0 == kNegInf) ? 1.f : exp2f(st.m0 - mn0);
-    const float c1 = (mn1 == kNegInf) ? 1.f : exp2f(st.m1 - mn1);
-    const float p0 = (mn0 == kNegInf) ? 0.f : exp2f(x0 - mn0);
-    const float p1 = (mn1 == kNegInf) ? 0.f : exp2f(x1 - mn1);
-    const float p2 = (mn0 == kNegInf) ? 0.f : exp2f(x2 - mn0);
-    const float p3 = (mn1 == kNegInf) ? 0.f : exp2f(x3 - mn1);
-    st.m0 = mn0;
-    st.m1 = mn1;
-    const uint32_t plo = pack_bf16x2(p0, p1), phi = pack_bf16x2(p2, p3);
-    st.l0 = fmaf(st.l0, c0, bf16_lo(plo) + bf16_lo(phi));
-    st.l1 = fmaf(st.l1, c1, bf16_hi(plo) + bf16_hi(phi));
-#pragma unroll
-    for (int tt = 0; tt < 8; ++tt) {
-        st.o[tt][0] *= c0; st.o[tt][1] *= c1;
-        st.o[tt][2] *= c0; st.o[tt][3] *= c1;
-    }
-    const uint32_t pb[2] = {movmatrix_trans(plo), movmatrix_trans(phi)};
-    // ---- O^T (128 dims x 8 heads) += V^T P^T ----
-    const bool partial = (int64_t)lb * kBlock + kBlock > L;
-#pragma unroll
-    for (int bx = 0; bx < 2; ++bx) {
-        const uint8_t *vb = t + (2 + bx) * kBoxBytes;
-        uint4 v0 = lds128(vb + (vt0 + 0) * 128 + off0);
-        uint4 v1 = lds128(vb + (vt0 + 4) * 128 + off1);
-        uint4 v2 = lds128(vb + (vt0 + 8) * 128 + off0);
-        uint4 v3 = lds128(vb + (vt0 + 12) * 128 + off1);
-        if (partial) {  // rows at or beyond L hold stale bits: keep them out of 0 * x
-            const int64_t b0 = (int64_t)lb * kBlock + vt0;
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            if (b0 >= L) v0 = z;
-            if (b0 + 4 >= L) v1 = z;
-            if (b0 + 8 >= L) v2 = z;
-            if (b0 + 12 >= L) v3 = z;
-        }
-#pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-            const uint32_t x = word(v0, wi), y = word(v1, wi);
-            const uint32_t x2 = word(v2, wi), y2 = word(v3, wi);
-            const uint32_t a[4] = {__byte_perm(x, y, 0x5410), __byte_perm(x, y, 0x7632),
-                                   __byte_perm(x2, y2, 0x5410), __byte_perm(x2, y2, 0x7632)};
-            mma_16816(st.o[4 * bx + wi], a, pb);
-        }
-    }
-}
-
-__device__ __forceinline__ void store_bf16(uint16_t *dst, float v) {
-    __nv_bfloat16 b = __float2bfloat16_rn(v);
-    *dst = *reinterpret_cast<uint16_t *>(&b);
-}
 }  // namespace
 
 size_t decode_smem_bytes(int32_t units, int stages) {
@@ -438,95 +305,22 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             const int32_t u_next = (seg_end < hi) ? find_unit(P, U, seg_end) : u;
 
             // ---- segment end: fold group 0 into group 1 lane by lane, merge the four warps ----
-            float l0 = st.l0, l1 = st.l1;
-#pragma unroll
-            for (int sh = 4; sh < 32; sh <<= 1) {
-                l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, sh);
-                l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, sh);
-            }
-            float *mine = scratch + wq * kScr;
-            float *oo = mine + 2 * kMaxG;
-            if (grp == 0) {
-                if (r == 0) {
-                    mine[2 * c] = st.m0; mine[2 * c + 1] = st.m1;
-                    mine[kMaxG + 2 * c] = l0; mine[kMaxG + 2 * c + 1] = l1;
-                }
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    const int psi = 64 * (t >> 2) + 8 * sig + 2 * (t & 3);
-                    oo[(2 * c) * kHS + swz(psi)] = st.o[t][0];
-                    oo[(2 * c + 1) * kHS + swz(psi)] = st.o[t][1];
-                    oo[(2 * c) * kHS + swz(psi + 1)] = st.o[t][2];
-                    oo[(2 * c + 1) * kHS + swz(psi + 1)] = st.o[t][3];
-                }
-            }
-            consumer_sync();
-            if (grp == 1) {
-                const float ma0 = mine[2 * c], ma1 = mine[2 * c + 1];
-                const float la0 = mine[kMaxG + 2 * c], la1 = mine[kMaxG + 2 * c + 1];
-                const float M0 = fmaxf(ma0, st.m0), M1 = fmaxf(ma1, st.m1);
-                const float fa0 = (ma0 == kNegInf) ? 0.f : exp2f(ma0 - M0);
-                const float fa1 = (ma1 == kNegInf) ? 0.f : exp2f(ma1 - M1);
-                const float fb0 = (st.m0 == kNegInf) ? 0.f : exp2f(st.m0 - M0);
-                const float fb1 = (st.m1 == kNegInf) ? 0.f : exp2f(st.m1 - M1);
-                float om[8][4];
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    const int psi = 64 * (t >> 2) + 8 * sig + 2 * (t & 3);
-                    om[t][0] = fmaf(fa0, oo[(2 * c) * kHS + swz(psi)], fb0 * st.o[t][0]);
-                    om[t][1] = fmaf(fa1, oo[(2 * c + 1) * kHS + swz(psi)], fb1 * st.o[t][1]);
-                    om[t][2] = fmaf(fa0, oo[(2 * c) * kHS + swz(psi + 1)], fb0 * st.o[t][2]);
-                    om[t][3] = fmaf(fa1, oo[(2 * c + 1) * kHS + swz(psi + 1)], fb1 * st.o[t][3]);
-                }
-                __syncwarp();  // every lane has read m, l before lanes r == 0 overwrite them
-                if (r == 0) {
-                    mine[2 * c] = M0; mine[2 * c + 1] = M1;
-                    mine[kMaxG + 2 * c] = fmaf(fa0, la0, fb0 * l0);
-                    mine[kMaxG + 2 * c + 1] = fmaf(fa1, la1, fb1 * l1);
-                }
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    const int psi = 64 * (t >> 2) + 8 * sig + 2 * (t & 3);
-                    oo[(2 * c) * kHS + swz(psi)] = om[t][0];
-                    oo[(2 * c + 1) * kHS + swz(psi)] = om[t][1];
-                    oo[(2 * c) * kHS + swz(psi + 1)] = om[t][2];
-                    oo[(2 * c + 1) * kHS + swz(psi + 1)] = om[t][3];
-                }
-            }
-            consumer_sync();
+            fold_groups(st, scratch, grp, wq, r, c, sig);
             if (seg_end < hi) load_unit(u_next);  // in flight while the merge runs
             const int nout = p.G * kD;
             uint16_t *out = p.out + (int64_t)u * p.G * kD;
             float *part = p.part + ((int64_t)cta * 2 + slot) * kPartFloats;
             for (int idx = ctid; idx < nout; idx += kConsThreads) {
                 const int h = idx >> 7, d = idx & (kD - 1);
-                float M = kNegInf;
-#pragma unroll
-                for (int w = 0; w < kDecW; ++w) M = fmaxf(M, scratch[w * kScr + h]);
-                float acc = 0.f, lsum = 0.f;
-#pragma unroll
-                for (int w = 0; w < kDecW; ++w) {
-                    const float mw = scratch[w * kScr + h];
-                    const float f = (mw == kNegInf) ? 0.f : exp2f(mw - M);
-                    acc = fmaf(f, scratch[w * kScr + 2 * kMaxG + h * kHS + swz(d)], acc);
-                    lsum = fmaf(f, scratch[w * kScr + kMaxG + h], lsum);
-                }
+                float M, acc, lsum;
+                merged_state(scratch, h, d, M, acc, lsum);
                 if (whole && p.mode == kModeResident) {
-                    float *rp = p.res_part + (int64_t)u * kPartFloats;
-                    rp[2 * kMaxG + h * kD + d] = acc;
-                    if (d == 0) {
-                        rp[h] = M;
-                        rp[kMaxG + h] = lsum;
-                    }
+                    store_partial(p.res_part + (int64_t)u * kPartFloats, h, d, M, acc, lsum);
                 } else if (whole) {
                     if (p.mode == kModeRest) merge_resident(p, u, h, d, M, acc, lsum);
                     store_bf16(out + idx, lsum > 0.f ? acc / lsum : 0.f);
                 } else {
-                    part[2 * kMaxG + h * kD + d] = acc;
-                    if (d == 0) {
-                        part[h] = M;
-                        part[kMaxG + h] = lsum;
-                    }
+                    store_partial(part, h, d, M, acc, lsum);
                 }
             }
             if (!whole) {
@@ -539,136 +333,29 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 if (ctid == 0) s_last = ((int32_t)atom_add_acq_rel_gpu(p.counter + u, 1u) == cl - cf);
                 consumer_sync();
                 if (s_last && C > 0 && C <= kOnePassPieces) {
-                    // last piece of the unit: merge the C pieces' partials (piece order) in one
-                    // pass, every thread loading what its 4 dims need at once
+                    // last piece of the unit: merge the C pieces' partials (piece t: slot 0 of CTA
+                    // cf + t) in one pass, every thread loading what its 4 dims need at once
                     if (ctid == 0) p.counter[u] = 0;
-                    for (int v = ctid; v < p.G * (kD / 4); v += kConsThreads) {
-                        const int h = v / (kD / 4), d4 = (v % (kD / 4)) * 4;
-                        const float *src0 = p.part + (int64_t)cf * 2 * kPartFloats;  // piece t: slot 0 of CTA cf + t
-                        float mt[kOnePassPieces];
-                        float ls = 0.f;
-                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (C <= kFewPieces) {
-                            // few pieces (C = 2 at the configs' sizes): every load at once, one round trip
-                            float lt[kFewPieces];
-                            float4 ot[kFewPieces];
-#pragma unroll
-                            for (int t = 0; t < kFewPieces; ++t) {
-                                const float *st_t = src0 + (int64_t)t * 2 * kPartFloats;
-                                mt[t] = t < C ? __ldcg(st_t + h) : kNegInf;
-                                lt[t] = t < C ? __ldcg(st_t + kMaxG + h) : 0.f;
-                                ot[t] = t < C ? __ldcg(reinterpret_cast<const float4 *>(st_t + 2 * kMaxG + h * kD + d4))
-                                              : make_float4(0.f, 0.f, 0.f, 0.f);
-                            }
-                            float M = kNegInf;
-#pragma unroll
-                            for (int t = 0; t < kFewPieces; ++t) M = fmaxf(M, mt[t]);
-#pragma unroll
-                            for (int t = 0; t < kFewPieces; ++t) {
-                                if (t < C) {
-                                    const float f = (mt[t] == kNegInf) ? 0.f : exp2f(mt[t] - M);
-                                    ls = fmaf(f, lt[t], ls);
-                                    acc.x = fmaf(f, ot[t].x, acc.x); acc.y = fmaf(f, ot[t].y, acc.y);
-                                    acc.z = fmaf(f, ot[t].z, acc.z); acc.w = fmaf(f, ot[t].w, acc.w);
-                                }
-                            }
-                        } else {
-#pragma unroll
-                            for (int t = 0; t < kOnePassPieces; ++t)
-                                mt[t] = t < C ? __ldcg(src0 + (int64_t)t * 2 * kPartFloats + h) : kNegInf;
-                            float M = kNegInf;
-#pragma unroll
-                            for (int t = 0; t < kOnePassPieces; ++t) M = fmaxf(M, mt[t]);
-#pragma unroll
-                            for (int t = 0; t < kOnePassPieces; ++t) {
-                                if (t < C) {
-                                    const float *st_t = src0 + (int64_t)t * 2 * kPartFloats;
-                                    const float f = (mt[t] == kNegInf) ? 0.f : exp2f(mt[t] - M);
-                                    const float4 o4 = __ldcg(reinterpret_cast<const float4 *>(st_t + 2 * kMaxG + h * kD + d4));
-                                    ls = fmaf(f, __ldcg(st_t + kMaxG + h), ls);
-                                    acc.x = fmaf(f, o4.x, acc.x); acc.y = fmaf(f, o4.y, acc.y);
-                                    acc.z = fmaf(f, o4.z, acc.z); acc.w = fmaf(f, o4.w, acc.w);
-                                }
-                            }
-                        }
-                        uint2 pk;
-                        if (ls > 0.f) {
-                            pk.x = pack_bf16x2(acc.x / ls, acc.y / ls);
-                            pk.y = pack_bf16x2(acc.z / ls, acc.w / ls);
-                        } else {
-                            pk.x = pk.y = 0u;
-                        }
-                        *reinterpret_cast<uint2 *>(out + h * kD + d4) = pk;
-                    }
+                    merge_pieces_onepass(p.part + (int64_t)cf * 2 * kPartFloats, 2 * kPartFloats, C, p.G, out, ctid);
                 } else if (s_last) {
                     // last contributor: merge the unit's partials in CTA order
                     if (ctid == 0) p.counter[u] = 0;
                     // the CTA partials (and, merging the rest pass, the resident state)
                     const int nc = cl - cf + 1 + (p.mode == kModeRest ? 1 : 0);  // <= Ge + 1
-                    float *fac = scratch;                               // [nc][8] scale of each partial
-                    float *lsum = fac + nc * kMaxG;                     // [8] merged denominators
-                    float *Ms = lsum + kMaxG;                           // [8] merged maxima
-                    const float **src = reinterpret_cast<const float **>(
-                        scratch + ((nc * kMaxG + 2 * kMaxG + 1) & ~1));  // [nc] partial states
+                    const MergeScratch ms = merge_scratch(scratch, nc);
                     for (int t = ctid; t < nc; t += kConsThreads) {
                         const int32_t cc = cf + t;
                         if (cc > cl) {
-                            src[t] = p.res_part + (int64_t)u * kPartFloats;
+                            ms.src[t] = p.res_part + (int64_t)u * kPartFloats;
                         } else {
                             const int sl = (C > 0 || find_unit(P, U, (int64_t)cc * W / Ge) == u) ? 0 : 1;
-                            src[t] = p.part + (int64_t)(cc * 2 + sl) * kPartFloats;
+                            ms.src[t] = p.part + (int64_t)(cc * 2 + sl) * kPartFloats;
                         }
                     }
                     consumer_sync();
-                    for (int h = warp; h < p.G; h += kConsWarps) {  // one warp per head
-                        float M = kNegInf;
-                        for (int t = lane; t < nc; t += 32) M = fmaxf(M, __ldcg(src[t] + h));
-#pragma unroll
-                        for (int sh = 16; sh > 0; sh >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, sh));
-                        float ls = 0.f;
-                        for (int t = lane; t < nc; t += 32) {
-                            const float mc = __ldcg(src[t] + h);
-                            const float f = (mc == kNegInf) ? 0.f : exp2f(mc - M);
-                            fac[t * kMaxG + h] = f;
-                            ls = fmaf(f, __ldcg(src[t] + kMaxG + h), ls);
-                        }
-#pragma unroll
-                        for (int sh = 16; sh > 0; sh >>= 1) ls += __shfl_xor_sync(0xFFFFFFFFu, ls, sh);
-                        if (lane == 0) {
-                            lsum[h] = ls;
-                            Ms[h] = M;
-                        }
-                    }
-                    consumer_sync();
-                    for (int v = ctid; v < p.G * (kD / 4); v += kConsThreads) {  // 4 dims per thread
-                        const int h = v / (kD / 4), d4 = (v % (kD / 4)) * 4;
-                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-                        for (int t = 0; t < nc; ++t) {
-                            const float f = fac[t * kMaxG + h];
-                            const float4 o4 = __ldcg(reinterpret_cast<const float4 *>(src[t] + 2 * kMaxG + h * kD + d4));
-                            acc.x = fmaf(f, o4.x, acc.x); acc.y = fmaf(f, o4.y, acc.y);
-                            acc.z = fmaf(f, o4.z, acc.z); acc.w = fmaf(f, o4.w, acc.w);
-                        }
-                        const float ls = lsum[h];
-                        if (p.mode == kModeResident) {  // the unit's state, for the rest pass
-                            float *rp = p.res_part + (int64_t)u * kPartFloats;
-                            *reinterpret_cast<float4 *>(rp + 2 * kMaxG + h * kD + d4) = acc;
-                            if (d4 == 0) {
-                                rp[h] = Ms[h];
-                                rp[kMaxG + h] = ls;
-                            }
-                            continue;
-                        }
-                        uint2 pk;
-                        if (ls > 0.f) {
-                            pk.x = pack_bf16x2(acc.x / ls, acc.y / ls);
-                            pk.y = pack_bf16x2(acc.z / ls, acc.w / ls);
-                        } else {
-                            pk.x = pk.y = 0u;
-                        }
-                        *reinterpret_cast<uint2 *>(out + h * kD + d4) = pk;
-                    }
+                    merge_general(ms, nc, p.G, out,
+                                  p.mode == kModeResident ? p.res_part + (int64_t)u * kPartFloats : nullptr, warp,
+                                  lane, ctid);
                 }
             }
             consumer_sync();  // scratch and s_last are reused by the next segment

@@ -104,10 +104,32 @@ struct DecodeParams {
 
 constexpr int kPartFloats = 2 * kMaxG + kMaxG * kD;  // m[8], l[8], o[8][128]
 
+// The fused step (nosa_fused_step): append + select + sparse decode of a device-resident store in
+// one launch, a team of C CTAs per unit.  Decode fields: q, e, seq_len, out, err, max_ctx,
+// blocks_per_unit (nblk), max_sel, G, units, qk_log2, pieces (C), k_e, k_q, nblk; part holds one
+// record per CTA, counter counts a unit's finished pieces.
+struct StepParams {
+    DecodeParams d;
+    AppendParams ap;          // T = 1
+    const void *ck;           // [u][nsub][D] fp32, or bf16 when ck_bf16
+    const int32_t *gamma_e;   // [u][k_e], read after the unit's append
+    const int32_t *gamma_n;   // [u]
+    int32_t *sel;             // [u][max_sel] out
+    int32_t *nsel;            // [u] out
+    int32_t *gq;              // [u][k_q] out or null
+    uint64_t *part_keys;      // [u][C][32] workspace: each team CTA's top-32 list
+    int32_t *score_ctr;       // [u] workspace: team CTAs that published their list
+    int32_t *ready;           // [u][2] workspace: 1 = the append is done, 1 = Gamma_q is known
+    int32_t *rest;            // [u][k_q] workspace: Gamma_q \ Gamma_e in rank order, -1 padded
+    int32_t nsub, ck_bf16;
+    float scale;
+};
+
 int launch_append(const AppendParams &p, cudaStream_t stream);
 int launch_select(const SelectParams &p, cudaStream_t stream);
 int launch_cache_sync(const CacheParams &p, cudaStream_t stream);
 int launch_decode(const DecodeParams &p, const CUtensorMap &tmap, cudaStream_t stream);
+int launch_step(const StepParams &p, const CUtensorMap &tmap, cudaStream_t stream);
 
 // The argument checks of nosa_select (config, state, pointers, workspace), with
 // nothing launched: NOSA_OK or the code nosa_select would return before a launch.
@@ -117,6 +139,10 @@ int select_args_ok(const nosa_config *c, const nosa_state *st, const uint16_t *q
 // Launch geometry, shared by the launchers and the workspace-size queries.
 int select_chunk_blocks(int32_t units, int32_t nblk, bool ck_bf16);
 int decode_ctas();
+// CTAs per unit of the fused step: as many as fit on the SMs at one CTA per SM (at most one per
+// decode item), or 1 when the units alone fill the GPU.
+int step_team_size(int32_t units, int32_t max_sel);
+size_t step_smem_bytes(int32_t nblk);
 constexpr int kMaxUnits = 2048;  // (seq, kv head) units per call: the decode kernel's prefix sums live in shared memory
 
 constexpr int kNumSms = 148;

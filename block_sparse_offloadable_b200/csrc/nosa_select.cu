@@ -58,30 +58,6 @@ __device__ __forceinline__ void sel_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kSelW * 32) : "memory");
 }
 
-// This lane's 4 dims of one pooled-key row in shared memory.
-__device__ __forceinline__ float4 row4(const uint8_t *tile, int row, int lane, float *) {
-    return lds128f(tile + row * (kD * 4) + lane * 16);
-}
-__device__ __forceinline__ float4 row4(const uint8_t *tile, int row, int lane, __nv_bfloat16 *) {
-    uint2 w;
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
-                 : "=r"(w.x), "=r"(w.y)
-                 : "r"(smem_u32(tile + row * (kD * 2) + lane * 8)));
-    return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
-}
-
-// One level of the transpose-reduction: lanes exchange the half they do not keep.
-template <int N>
-__device__ __forceinline__ void reduce_level(float (&v)[32], int lane, int o) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-        const float send = upper ? v[i] : v[i + N];
-        const float keep = upper ? v[i + N] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
-    }
-}
-
 // Fill reading, one warp: Gamma_e = the first k_e pool entries (E rank order)
 // outside Gamma_q, whose bits are already set in `bitmap`; their bits are set
 // too, then the pool keeps only the entries in Sel = Gamma_q + Gamma_e, in

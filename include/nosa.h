@@ -8,7 +8,8 @@
  *   nosa_select           two-stage block scores, Gamma_q, union with Gamma_e and local
  *   nosa_cache_sync       (offload mode) swap blocks: fetch misses host -> device cache
  *   nosa_sparse_decode    exact softmax attention over the selected blocks
- * or three, with nosa_append_select doing the first two in one launch.  Also:
+ * or three, with nosa_append_select doing the first two in one launch; with the KV
+ * store in device memory, nosa_fused_step does the whole step in one launch.  Also:
  * nosa_compress_append_head (the eviction logits from the fused eviction head),
  * nosa_decode_resident + nosa_decode_rest (the attention split around the
  * select and the cache sync), nosa_dense_decode (the full-attention
@@ -165,7 +166,8 @@ enum nosa_call {
     NOSA_WS_SPARSE_DECODE = 1,
     NOSA_WS_DENSE_DECODE = 2,
     NOSA_WS_CACHE_SYNC = 3,
-    NOSA_WS_SPLIT = 4  /* the buffer nosa_decode_resident fills and nosa_decode_rest reads */
+    NOSA_WS_SPLIT = 4,  /* the buffer nosa_decode_resident fills and nosa_decode_rest reads */
+    NOSA_WS_FUSED_STEP = 5
 };
 
 /* Validate a configuration: NOSA_OK or a negative code. */
@@ -280,6 +282,32 @@ int nosa_select(const nosa_config *cfg, const nosa_state *st, const uint16_t *q,
 int nosa_append_select(const nosa_config *cfg, const nosa_state *st, const uint16_t *k_new,
                        const uint16_t *v_new, const float *e_new, const uint16_t *q, int32_t *sel,
                        int32_t *nsel, int32_t *gq, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * a1 (decode, T = 1) + a2 + a3 + a5 in one launch, for a KV store in device
+ * memory: nosa_append_select followed by nosa_sparse_decode, with the same
+ * arguments, results and device errors (out equal up to the order of
+ * floating-point sums), but one kernel.  NOSA pages: as those calls; the
+ * overlap follows from the dual selection (gist.science summary of
+ * 2510.13602, "Mecanisme de double selection"; montaan.com "Key Design
+ * Components" item 4): Gamma_e needs no query, so its blocks and the local
+ * block are attended while the query-aware scores are being computed, and only
+ * the blocks of Gamma_q outside Gamma_e wait for the selection.
+ *
+ *   k_new, v_new, e_new, q, sel, nsel, gq   as nosa_append_select
+ *   out   device bf16 [B][Hq][D] out, as nosa_sparse_decode
+ *   ws    device workspace of nosa_workspace_bytes(cfg, NOSA_WS_FUSED_STEP) bytes
+ *
+ * Each unit is served by a team of CTAs that wait on one another (bounded
+ * waits); with several CTAs per unit the kernel is launched cooperatively, so
+ * the whole grid (at most one CTA per SM) must be able to run at once:
+ * NOSA_ERR_CUDA if it cannot.  NOSA_ERR_UNSUPPORTED with offload == 1 (the
+ * cache sync runs between the selection and the decode) or NOSA_FLAG_FILL
+ * (Gamma_e is formed after Gamma_q there).
+ */
+int nosa_fused_step(const nosa_config *cfg, const nosa_state *st, const uint16_t *k_new, const uint16_t *v_new,
+                    const float *e_new, const uint16_t *q, int32_t *sel, int32_t *nsel, int32_t *gq, uint16_t *out,
+                    void *ws, size_t ws_bytes, void *stream);
 
 /*
  * a4 -- block cache synchronisation (offload mode).  NOSA pages: montaan.com

@@ -29,7 +29,7 @@ MAX_ABS, MEAN_ABS, REL_L2 = 1e-2, 1e-3, 1e-2
 class Scenario:
     def __init__(self, B, Hq, Hkv, k_q, k_e, L0, steps, offload=False, seed=0, layer=0, lens=None,
                  max_ctx=None, dense=False, ck_bf16=False, fill=False, head=False, split=False, fused=False,
-                 layer_step=False):
+                 layer_step=False, step=False):
         self.B, self.Hq, self.Hkv, self.k_q, self.k_e = B, Hq, Hkv, k_q, k_e
         self.G = Hq // Hkv
         self.units = B * Hkv
@@ -44,6 +44,7 @@ class Scenario:
         self.split = split  # decode_resident on a side stream during select / cache_sync, then decode_rest
         self.fused = fused  # decode steps append and select in one launch (nosa_append_select)
         self.layer_step = layer_step  # decode steps through NosaLayer.decode_step (the documented one-call step)
+        self.step = step  # decode steps through nosa_fused_step (append, select and decode in one launch)
         self.W = synth.head_weights(seed, layer, Hkv) if head else None
 
     def cfg(self):
@@ -112,7 +113,9 @@ def run_gpu(sc, data):
         en = torch.from_numpy(np.ascontiguousarray(E[np.arange(sc.units), idx][:, None])).cuda()
         q = _dev16(Q[t])
         out = torch.empty((sc.B, sc.Hq, 128), dtype=torch.int16, device="cuda")
-        if sc.layer_step:
+        if sc.step:
+            lay.fused_step(kn, vn, en, q, out)
+        elif sc.layer_step:
             lay.decode_step(kn, vn, en, q, out)
         elif sc.fused:
             lay.append_select(kn, vn, en, q)
@@ -122,14 +125,14 @@ def run_gpu(sc, data):
             cur = torch.cuda.current_stream()
             side.wait_stream(cur)
             lay.decode_resident(q, side)
-        if not (sc.fused or sc.layer_step):
+        if not (sc.fused or sc.layer_step or sc.step):
             lay.select(q)
         if sc.offload and not sc.layer_step:
             lay.cache_sync()
         if sc.split:
             cur.wait_stream(side)
             lay.decode_rest(q, out)
-        elif not sc.layer_step:
+        elif not (sc.layer_step or sc.step):
             lay.sparse_decode(q, out)
         res["sel"].append(lay.sel.cpu().numpy())
         res["nsel"].append(lay.nsel.cpu().numpy())

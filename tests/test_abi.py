@@ -115,3 +115,41 @@ def test_workspace_sizes_follow_the_launch_geometry(L, bf16):
 def test_strerror(L):
     for code in (0, -1, -2, -3, -4, -5, -6, -7, -99):
         assert isinstance(L.nosa_strerror(code), bytes)
+
+
+def _team(units, max_sel, sms=148):
+    return 1 if units > sms else min(sms // units, max_sel)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_fused_step_workspace(L, bf16):
+    # per unit: two counters and two flags; per CTA (units x team size): a 32-key list and a partial
+    # state; per unit: k_q slots of Gamma_q outside Gamma_e
+    for batch, heads_kv, k_q, k_e in ((1, 1, 16, 48), (8, 2, 16, 48), (32, 2, 16, 48), (80, 2, 8, 24),
+                                      (2, 2, 32, 256), (4, 4, 0, 16)):
+        c = cfg(batch=batch, heads_q=heads_kv * 4, heads_kv=heads_kv, k_q=k_q, k_e=k_e, ck_bf16=bf16)
+        units, max_sel = batch * heads_kv, k_q + k_e + 1
+        ctas = units * _team(units, max_sel)
+        want = (_align256(units * 16) + _align256(ctas * 32 * 8) + _align256(ctas * (2 * 8 + 8 * 128) * 4) +
+                units * max(k_q, 1) * 4)
+        assert nosa.nosa_workspace_bytes(c, nosa.WS_FUSED_STEP) == want, (batch, heads_kv)
+    # not built for the offload store or the fill reading
+    assert nosa.nosa_workspace_bytes(cfg(offload=True), nosa.WS_FUSED_STEP) == 0
+    assert nosa.nosa_workspace_bytes(cfg(fill=True), nosa.WS_FUSED_STEP) == 0
+
+
+def test_fused_step_refuses_before_any_launch(L):
+    st = nosa.State()
+    P = ctypes.c_void_p
+
+    def call(c, e_new):
+        return L.nosa_fused_step(ctypes.byref(c), ctypes.byref(st), P(16), P(16), e_new, P(16), P(16), P(16), None,
+                                 P(16), None, 0, None)
+
+    assert call(cfg(offload=True), P(16)) == nosa.ERR_UNSUPPORTED
+    assert call(cfg(fill=True), P(16)) == nosa.ERR_UNSUPPORTED
+    assert call(cfg(), None) == nosa.ERR_ARG
+    assert call(cfg(), P(16)) == nosa.ERR_PTR  # the state's buffers are missing
+    bad = cfg()
+    bad.k_q = 33
+    assert call(bad, P(16)) == nosa.ERR_UNSUPPORTED

@@ -33,6 +33,8 @@ MODES = {
     "offload-separate": dict(offload=True),
     "layer-step": dict(layer_step=True, offload=True),
     "ck-bf16": dict(fused=True, ck_bf16=True),
+    "fused-step": dict(step=True),
+    "fused-step-bf16": dict(step=True, ck_bf16=True),
 }
 
 
@@ -87,7 +89,7 @@ def test_golden_fixture(name, mode):
     check_expected(sc, gpu, 0, spec, spec["k_q"])
 
 
-@pytest.mark.parametrize("mode", ["separate", "fused", "offload"])
+@pytest.mark.parametrize("mode", ["separate", "fused", "offload", "fused-step"])
 def test_golden_tie_two_way_order(mode):
     """Both tied blocks taken (k_q = 2): Gamma_q lists them in rank order, the lower index first."""
     spec = dict(cases.load_fixture("tie_lower_index.json"), k_q=2)
@@ -155,12 +157,22 @@ TIE_CASES = {
     "fill-offload": dict(B=2, Hq=8, Hkv=2, k_q=8, k_e=3, L0=64 * 30 + 9, steps=40, offload=True, fill=True),
     "ck-bf16": dict(B=2, Hq=16, Hkv=2, k_q=4, k_e=12, L0=64 * 37 + 21, steps=40, fused=True, ck_bf16=True),
     "split": dict(B=2, Hq=16, Hkv=2, k_q=4, k_e=12, L0=64 * 40 + 3, steps=30, offload=True, split=True),
+    "fused-step": dict(B=2, Hq=16, Hkv=2, k_q=4, k_e=12, L0=64 * 37 + 21, steps=40, step=True),
+    "fused-step-bf16": dict(B=2, Hq=16, Hkv=2, k_q=4, k_e=12, L0=64 * 37 + 21, steps=40, step=True, ck_bf16=True),
+    "fused-step-mha": dict(B=1, Hq=4, Hkv=4, k_q=4, k_e=12, L0=64 * 20, steps=66, step=True),
+    "fused-step-budget-edge": dict(B=1, Hq=16, Hkv=2, k_q=32, k_e=96, L0=64 * 300 + 11, steps=6, step=True),
 }
+
+
+def _tie_seed(name):
+    # the fused-step cases come after the others, whose seeds stay as they were
+    base = sorted(n for n in TIE_CASES if not n.startswith("fused-step"))
+    return 40 + base.index(name) if name in base else 70 + sorted(TIE_CASES).index(name)
 
 
 @pytest.mark.parametrize("name", sorted(TIE_CASES))
 def test_exact_ties(name):
-    sc = H.Scenario(seed=40 + sorted(TIE_CASES).index(name), **TIE_CASES[name])
+    sc = H.Scenario(seed=_tie_seed(name), **TIE_CASES[name])
     data = tie_data(sc, seed=sc.seed)
     _, st = run_exact(sc, data)
     H.record_stats(f"ties {name}", st)
