@@ -36,17 +36,21 @@ import synth  # noqa: E402
 METRIC = "sparse decode tokens/s/GPU at 128K ctx; % of HBM and PCIe roofline"
 D = 128
 
-# Every workload runs the decode-time append fused into the select launch (nosa_append_select);
-# --unfused launches them separately.
+# Device-store workloads run each layer's step in one launch (nosa_fused_step; --no-fused-step: the
+# two-launch path); the offload workload runs the decode-time append fused into the select launch
+# (nosa_append_select), then the cache sync and the decode.  --unfused launches append and select
+# separately (and turns the fused step off).
 WORKLOADS = {
     # one layer, batch 1, 16 q / 16 kv heads, 8K context, 32 decode steps, KV in device memory
-    "mha-8k": dict(layers=1, B=1, Hq=16, Hkv=16, L=8192, k_q=16, k_e=48, steps=32, offload=False, fuse=True),
+    "mha-8k": dict(layers=1, B=1, Hq=16, Hkv=16, L=8192, k_q=16, k_e=48, steps=32, offload=False, fuse=True,
+                   step=True),
     # one layer, batch 8, GQA 16 q / 2 kv heads, 16K context, 128 decode steps, KV in device memory
-    "gqa-16k": dict(layers=1, B=8, Hq=16, Hkv=2, L=16384, k_q=16, k_e=48, steps=128, offload=False, fuse=True),
+    "gqa-16k": dict(layers=1, B=8, Hq=16, Hkv=2, L=16384, k_q=16, k_e=48, steps=128, offload=False, fuse=True,
+                    step=True),
     # 28-layer stack, batch 32, GQA 16/2, 32K context, 64 decode steps, KV in device memory
     # (its line also carries the library's dense decode on the same inputs)
     "stack28-32k": dict(layers=28, B=32, Hq=16, Hkv=2, L=32768, k_q=16, k_e=48, steps=64, offload=False, fuse=True,
-                        dense_compare=True),
+                        step=True, dense_compare=True),
     # 28-layer stack, batch 64, GQA 16/2, 128K context, 256 decode steps, KV in pinned host memory
     "offload28-128k": dict(layers=28, B=64, Hq=16, Hkv=2, L=131072, k_q=16, k_e=48, steps=256, offload=True, fuse=True),
 }
@@ -69,7 +73,9 @@ def describe(c, groups):
         s += ", eviction logits from the fused synthetic eviction head"
     if c.get("split"):
         s += ", decode split: Gamma_e + local attended while select and the cache sync run"
-    if c.get("fuse"):
+    if c.get("step") and not (c["offload"] or c.get("fill") or c.get("head") or c.get("split")):
+        s += ", each layer's step (append, select, decode) in one launch"
+    elif c.get("fuse"):
         s += ", append and select fused in one launch"
     return s
 
@@ -982,7 +988,7 @@ def run_sweep(args, dev):
     for L in SWEEP["context"]:
         for B in SWEEP["batch"]:
             base = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=16, k_e=48, steps=3 + warmup + steps,
-                        ck_bf16=args.ck_bf16, fuse=not args.unfused)
+                        ck_bf16=args.ck_bf16, fuse=not args.unfused, step=not (args.unfused or args.no_fused_step))
             dense = Workload(dict(base, offload=False), 3 + warmup + steps + 1, seed=args.seed, dense=True,
                              device=dev)
             dense_ms, _ = dense.time_steps(warmup, steps)
@@ -1084,8 +1090,9 @@ def main():
                     help="compute the eviction logits with the fused synthetic eviction head inside append")
     ap.add_argument("--unfused", action="store_true",
                     help="launch the decode-time append and the select separately (default: one launch)")
-    ap.add_argument("--fused-step", action="store_true",
-                    help="device store: the whole step of a layer (append, select, decode) in one launch")
+    ap.add_argument("--no-fused-step", action="store_true",
+                    help="device store: append + select, then decode (two launches) instead of the whole step "
+                         "of a layer in one launch")
     ap.add_argument("--split", action="store_true",
                     help="split decode: attend Gamma_e + the local block while select and the cache sync run")
     ap.add_argument("--fill", action="store_true",
@@ -1102,8 +1109,9 @@ def main():
         c["split"] = True
     if args.unfused:
         c["fuse"] = False
-    if args.fused_step:
-        c["step"] = True
+        c["step"] = False
+    if args.no_fused_step:
+        c["step"] = False
     if args.layers is not None:
         c["layers"] = args.layers
     world = int(os.environ.get("WORLD_SIZE", "1"))

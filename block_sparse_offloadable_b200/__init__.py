@@ -342,8 +342,12 @@ class NosaLayer:
         nosa_dense_decode(self.cfg, self.state, q, out, self.ws_dense, stream)
 
     def decode_step(self, k_new, v_new, e_new, q, out, stream=None):
-        """One decode step of this layer: append + select in one launch, the cache sync (offload),
-        and the sparse decode into `out` (bf16 bits [B][Hq][D])."""
+        """One decode step of this layer into `out` (bf16 bits [B][Hq][D]): with the KV store in
+        device memory and the union reading, nosa_fused_step (one launch); otherwise append +
+        select in one launch, the cache sync (offload), and the sparse decode."""
+        if self.ws_step is not None:
+            self.fused_step(k_new, v_new, e_new, q, out, stream)
+            return
         self.append_select(k_new, v_new, e_new, q, stream)
         if self.cfg.offload:
             self.cache_sync(stream)

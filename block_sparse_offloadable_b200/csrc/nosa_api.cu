@@ -126,8 +126,8 @@ int select_nchunks(const nosa_config *c, const Geo &g) {
 // Words of the per-unit block bitmap in the split-decode buffer.
 size_t split_bits_words(const Geo &g) { return (size_t)g.nblk / 32 + 1; }
 
-// Workspace of the fused step: [score counter, piece counter, 2 flags] per unit, then each team
-// CTA's top-32 list, each CTA's partial state, and each unit's Gamma_q \ Gamma_e list.
+// Workspace of the fused step: [launch count, piece counter, "appended" flag, spare] per unit, then
+// each team CTA's top-32 list, each CTA's partial state, and each unit's Gamma_q \ Gamma_e list.
 struct StepWs {
     int32_t C;
     size_t keys, parts, rest, total;
@@ -485,10 +485,10 @@ int nosa_fused_step(const nosa_config *c, const nosa_state *st, const uint16_t *
     sp.sel = sel;
     sp.nsel = nsel;
     sp.gq = c->k_q > 0 ? gq : nullptr;
-    sp.score_ctr = reinterpret_cast<int32_t *>(wb);
-    sp.ready = reinterpret_cast<int32_t *>(wb) + 2 * g.units;
+    sp.epoch = reinterpret_cast<int32_t *>(wb);
+    sp.appended = reinterpret_cast<int32_t *>(wb) + 2 * g.units;
     sp.part_keys = reinterpret_cast<uint64_t *>(wb + w.keys);
-    sp.rest = reinterpret_cast<int32_t *>(wb + w.rest);
+    sp.rest = reinterpret_cast<uint32_t *>(wb + w.rest);
     sp.nsub = (int32_t)g.nsub;
     sp.ck_bf16 = (c->flags & NOSA_FLAG_CK_BF16) != 0;
     sp.scale = c->scale;

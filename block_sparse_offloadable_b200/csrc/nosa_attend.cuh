@@ -257,20 +257,23 @@ __device__ __forceinline__ uint2 pack_out4(float4 acc, float ls) {
 
 // The last of C <= kOnePassPieces pieces of a unit merges their partial records, piece t at
 // src0 + t * stride, in piece order, in one pass: each consumer thread takes 4 dims of one head
-// and issues its loads at once (all of them with at most kFewPieces pieces).  Writes bf16 out.
+// and issues its loads at once (all of them with at most kAtOnce pieces: one round trip; more
+// registers).  Writes bf16 out.
+template <int kAtOnce = kFewPieces>
 __device__ __forceinline__ void merge_pieces_onepass(const float *src0, int64_t stride, int C, int G, uint16_t *out,
                                                      int ctid) {
+    static_assert(kAtOnce <= kOnePassPieces, "at most kOnePassPieces pieces");
     for (int v = ctid; v < G * (kD / 4); v += kConsThreads) {
         const int h = v / (kD / 4), d4 = (v % (kD / 4)) * 4;
         float mt[kOnePassPieces];
         float ls = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (C <= kFewPieces) {
+        if (C <= kAtOnce) {
             // few pieces: every load at once, one round trip
-            float lt[kFewPieces];
-            float4 ot[kFewPieces];
+            float lt[kAtOnce];
+            float4 ot[kAtOnce];
 #pragma unroll
-            for (int t = 0; t < kFewPieces; ++t) {
+            for (int t = 0; t < kAtOnce; ++t) {
                 const float *st_t = src0 + (int64_t)t * stride;
                 mt[t] = t < C ? __ldcg(st_t + h) : kNegInf;
                 lt[t] = t < C ? __ldcg(st_t + kMaxG + h) : 0.f;
@@ -279,9 +282,9 @@ __device__ __forceinline__ void merge_pieces_onepass(const float *src0, int64_t 
             }
             float M = kNegInf;
 #pragma unroll
-            for (int t = 0; t < kFewPieces; ++t) M = fmaxf(M, mt[t]);
+            for (int t = 0; t < kAtOnce; ++t) M = fmaxf(M, mt[t]);
 #pragma unroll
-            for (int t = 0; t < kFewPieces; ++t) {
+            for (int t = 0; t < kAtOnce; ++t) {
                 if (t < C) {
                     const float f = (mt[t] == kNegInf) ? 0.f : exp2f(mt[t] - M);
                     ls = fmaf(f, lt[t], ls);

@@ -117,10 +117,10 @@ struct StepParams {
     int32_t *sel;             // [u][max_sel] out
     int32_t *nsel;            // [u] out
     int32_t *gq;              // [u][k_q] out or null
-    uint64_t *part_keys;      // [u][C][32] workspace: each team CTA's top-32 list
-    int32_t *score_ctr;       // [u] workspace: team CTAs that published their list
-    int32_t *ready;           // [u][2] workspace: 1 = the append is done, 1 = Gamma_q is known
-    int32_t *rest;            // [u][k_q] workspace: Gamma_q \ Gamma_e in rank order, -1 padded
+    uint64_t *part_keys;      // [u][C][32] workspace: each team CTA's top-32 list, tagged
+    int32_t *epoch;           // [u] workspace: launches completed (tags this launch's lists and slots)
+    int32_t *appended;        // [u] workspace: 1 = this launch's append is done
+    uint32_t *rest;           // [u][k_q] workspace: Gamma_q \ Gamma_e in rank order, tagged
     int32_t nsub, ck_bf16;
     float scale;
 };

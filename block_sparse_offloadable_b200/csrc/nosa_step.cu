@@ -9,20 +9,26 @@
 // query-aware scores that decide Gamma_q are still being computed.
 //
 // Design.  Each unit (seq, kv head) has a team of C CTAs, one per SM (units * C <= the SM count,
-// or C = 1 when the units alone fill the GPU).  Team CTA c
-//  * (c = 0, on an extra warp) appends the token exactly as nosa_compress_append does and raises
-//    the unit's "appended" flag;
+// or C = 1 when the units alone fill the GPU).  A CTA has eight consumer warps, a producer warp
+// and a selection warp.  Team CTA c
+//  * (c = 0, selection warp) appends the token exactly as nosa_compress_append does and raises
+//    the unit's "appended" flag (a release store: the append wrote what other CTAs then read);
 //  * streams its 1/C share of the unit's candidate pooled keys through the stage ring, 16 blocks
-//    (fp32) or 32 (bf16) per 32 KiB stage, scores them (q_hat . kbar * scale, max over the four
-//    sub-blocks of a block) and keeps a top-32 list per warp; the team's last CTA to publish its
-//    list merges the C lists into Gamma_q, writes S(t) exactly as nosa_select does, writes the
-//    Gamma_q blocks outside Gamma_e in rank order, and raises the unit's "selected" flag;
-//  * attends piece c of the unit's decode list [Gamma_e (k_e slots) | local block | Gamma_q minus
-//    Gamma_e (k_q slots)] through the same ring, skipping empty slots: the producer waits for
-//    "appended" before its first item and for "selected" before the first Gamma_q item, which
-//    come last in the list;
+//    (fp32) or 32 (bf16) per 32 KiB stage; the consumers score them (q_hat . kbar * scale, max
+//    over the four sub-blocks of a block), keep a top-32 list per warp, hand the lists to the
+//    selection warp and go straight on to the attention;
+//  * (selection warp) merges the eight lists; team CTA 0 gathers the others' lists, merges them
+//    into Gamma_q, writes S(t) exactly as nosa_select does and writes the Gamma_q blocks outside
+//    Gamma_e in rank order;
+//  * attends its piece of the unit's decode slots: a 1/C share of the k_e + 1 slots of Gamma_e
+//    and the local block, then a 1/C share of the k_q slots of Gamma_q minus Gamma_e, through the
+//    same ring, skipping empty slots; the producer waits for "appended" before its first slot
+//    and, for each Gamma_q slot, until team CTA 0 has written it;
 //  * counts its piece; the unit's last piece merges the C partial states and writes the output,
-//    then clears the unit's flags and counters for the next launch.
+//    then clears the unit's flag and piece counter and counts the launch.
+// The lists and the Gamma_q slots pass between CTAs without fences: each 64- or 32-bit word
+// carries a tag of this launch (from the unit's launch count), and the reader polls until the tag
+// is current; a gpu-scope release in mid-stream waits for the SM's copies in flight (~2 us).
 // Stage s of the ring always belongs to consumer group s % 2, in both phases.  Every cross-CTA
 // wait is bounded and waits only for CTAs of the same team, which the cooperative launch keeps
 // resident together; a wait that runs out sets NOSA_EFLAG_TIMEOUT and the CTA drains.
@@ -35,18 +41,52 @@ namespace nosa {
 
 namespace {
 constexpr int kStepS = 6;                            // ring stages of 32 KiB (+ 256 B of logits)
-constexpr int kStepThreads = (kConsWarps + 2) * 32;  // consumers, the producer, the append warp
+constexpr int kStepThreads = (kConsWarps + 2) * 32;  // consumers, the producer, the selection warp
 constexpr int kProducerWarp = kConsWarps;
-constexpr int kAppendWarp = kConsWarps + 1;
+constexpr int kSelectWarp = kConsWarps + 1;
 static_assert(kStepS % kGroups == 0, "stage s must always be consumed by group s % kGroups");
 
-// The consumer warps and the append warp meet here before a team CTA publishes its list, so that
-// the append has read the old length before the finalizing CTA writes the new one.
-__device__ __forceinline__ void append_barrier_sync() {
-    asm volatile("bar.sync 2, %0;" ::"n"(kConsThreads + 32) : "memory");
+// Named barriers between the consumer warps and the selection warp (one side arrives, the other
+// waits): barrier 2, the consumers' lists are in shared memory; barrier 3, the selection warp is
+// done (so the flag it raised and its writes come before the CTA counts its piece).
+constexpr int kSelBarThreads = kConsThreads + 32;
+__device__ __forceinline__ void lists_arrive() { asm volatile("bar.arrive 2, %0;" ::"n"(kSelBarThreads) : "memory"); }
+__device__ __forceinline__ void lists_wait() { asm volatile("bar.sync 2, %0;" ::"n"(kSelBarThreads) : "memory"); }
+__device__ __forceinline__ void select_done_arrive() {
+    asm volatile("bar.arrive 3, %0;" ::"n"(kSelBarThreads) : "memory");
 }
-__device__ __forceinline__ void append_barrier_arrive() {
-    asm volatile("bar.arrive 2, %0;" ::"n"(kConsThreads + 32) : "memory");
+__device__ __forceinline__ void select_done_wait() { asm volatile("bar.sync 3, %0;" ::"n"(kSelBarThreads) : "memory"); }
+
+// Tagged words.  A list entry: the key's score order (32 bits), 0x3FFF - block (14 bits: blocks
+// < 2^14 at max_ctx <= 2^20) and the tag (18 bits); an empty entry is the tag alone.  A Gamma_q
+// slot: (block + 1) << 18 | tag, block -1 for an empty slot.  Tags run 1 .. 2^18 - 1.
+constexpr int kTagBits = 18;
+constexpr uint32_t kTagMask = (1u << kTagBits) - 1u;
+__device__ __forceinline__ uint32_t launch_tag(int32_t launches) { return ((uint32_t)launches % kTagMask) + 1u; }
+__device__ __forceinline__ uint64_t pack_key(uint64_t key, uint32_t tag) {
+    if (key == 0ull) return tag;
+    return (key & 0xFFFFFFFF00000000ull) | ((uint64_t)(0x3FFFu - (uint32_t)key_block(key)) << kTagBits) | tag;
+}
+__device__ __forceinline__ uint64_t unpack_key(uint64_t w) {
+    if ((w >> 32) == 0ull) return 0ull;
+    const uint32_t blk = 0x3FFFu - (uint32_t)((w >> kTagBits) & 0x3FFFu);
+    return (w & 0xFFFFFFFF00000000ull) | (uint64_t)(0xFFFFFFFFu - blk);
+}
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ void st_relaxed_u32(uint32_t *p, uint32_t v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // Pooled-key rows per consumer warp per stage: a stage is 32 KiB either way.
@@ -60,61 +100,39 @@ static_assert(stage_blocks<float>() * kSubPerBlock * kD * 4 == kBlockBytes, "a s
 static_assert(stage_blocks<__nv_bfloat16>() * kSubPerBlock * kD * 2 == kBlockBytes,
               "a score stage fills a ring stage");
 
-// The eight consumer warps' lists (lists[w * 32 + lane], warp w's in `list`) merged as a tree; the
-// result is in warp 0's `list`.  Called by every consumer thread.
-__device__ __forceinline__ void tree_merge(uint64_t &list, uint64_t *lists, int warp, int lane) {
-    lists[warp * 32 + lane] = list;
-    consumer_sync();
-    if (warp < 4) list_merge(list, lists[(warp + 4) * 32 + lane], lane);
-    if (warp < 4 && warp >= 2) lists[warp * 32 + lane] = list;
-    consumer_sync();
-    if (warp < 2) list_merge(list, lists[(warp + 2) * 32 + lane], lane);
-    if (warp == 1) lists[32 + lane] = list;
-    consumer_sync();
-    if (warp == 0) list_merge(list, lists[32 + lane], lane);
+// The best 32 keys of lists l[0..n), n <= 8, merged as a tree; the merges of one level are
+// independent, so their shuffle chains interleave.  Conditions are uniform over the warp.
+__device__ __forceinline__ uint64_t merge_lists(uint64_t (&l)[8], int n, int lane) {
+#pragma unroll
+    for (int w = 1; w < 8; w <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; i += 2 * w)
+            if (i + w < n) list_merge(l[i], l[i + w], lane);
+    }
+    return l[0];
 }
 
-// Warp 0 of the unit's finalizing CTA: Gamma_q from the merged list, S(t) = Gamma_q U Gamma_e U
-// {local} as nosa_select writes it, the Gamma_q blocks outside Gamma_e for the decode, the new
-// length; then the "selected" flag.
+// The selection warp of team CTA 0: Gamma_q from the merged list, S(t) = Gamma_q U Gamma_e U
+// {local} as nosa_select writes it, the Gamma_q blocks outside Gamma_e (tagged) for the decode, the
+// new length.  `bitmap` already holds Gamma_e over the words of the nb_c candidates.
 __device__ __forceinline__ void finalize_unit(const StepParams &sp, int32_t u, uint64_t list, int32_t L, int32_t nb_c,
-                                              bool grow, uint32_t *bitmap, int lane) {
+                                              bool grow, uint32_t *bitmap, uint32_t tag, int lane) {
     const DecodeParams &p = sp.d;
-    // Gamma_e as this step's append left it
-    int ok = 1;
-    if (lane == 0) ok = flag_wait(sp.ready + 2 * u);
-    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-    if (!ok && lane == 0) set_error(p.err, NOSA_EFLAG_TIMEOUT);
-    const int32_t ne = L > 0 ? min(max(__ldcg(sp.gamma_n + u), 0), p.k_e) : 0;
-    int32_t ge_reg[kMaxKe / 32];
-#pragma unroll
-    for (int i = 0; i < kMaxKe / 32; ++i) {
-        const int j = lane + 32 * i;
-        ge_reg[i] = (j < ne) ? __ldcg(sp.gamma_e + (int64_t)u * p.k_e + j) : -1;
-    }
     const int32_t myid = (lane < p.k_q && list != 0ull) ? key_block(list) : -1;
     if (sp.gq && lane < p.k_q) sp.gq[(int64_t)u * p.k_q + lane] = myid;
     int32_t *sel = sp.sel + (int64_t)u * p.max_sel;
-    int32_t *rest = sp.rest + (int64_t)u * p.k_q;
+    uint32_t *rest = sp.rest + (int64_t)u * p.k_q;
     if (L <= 0) {
         for (int i = lane; i < p.max_sel; i += 32) sel[i] = -1;
-        for (int i = lane; i < p.k_q; i += 32) rest[i] = -1;
+        for (int i = lane; i < p.k_q; i += 32) st_relaxed_u32(rest + i, tag);
         if (lane == 0) sp.nsel[u] = 0;
     } else {
         const int32_t nw = (nb_c + 31) >> 5;
-        for (int i = lane; i < nw; i += 32) bitmap[i] = 0;
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < kMaxKe / 32; ++i) {
-            const int32_t id = ge_reg[i];
-            if (id >= 0 && id < nb_c) atomicOr(&bitmap[id >> 5], 1u << (id & 31));
-        }
-        __syncwarp();
-        // Gamma_q blocks not in Gamma_e, in rank order: the decode list's last k_q slots
+        // Gamma_q blocks not in Gamma_e, in rank order: the decode's Gamma_q slots
         const bool fresh = myid >= 0 && myid < nb_c && !((bitmap[myid >> 5] >> (myid & 31)) & 1u);
         const unsigned m = __ballot_sync(0xFFFFFFFFu, fresh);
-        if (fresh) rest[__popc(m & ((1u << lane) - 1u))] = myid;
-        for (int i = __popc(m) + lane; i < p.k_q; i += 32) rest[i] = -1;
+        if (fresh) st_relaxed_u32(rest + __popc(m & ((1u << lane) - 1u)), ((uint32_t)(myid + 1) << kTagBits) | tag);
+        for (int i = __popc(m) + lane; i < p.k_q; i += 32) st_relaxed_u32(rest + i, tag);
         __syncwarp();  // every lane has tested its bit before the Gamma_q bits go in
         if (myid >= 0 && myid < nb_c) atomicOr(&bitmap[myid >> 5], 1u << (myid & 31));
         __syncwarp();
@@ -145,11 +163,8 @@ __device__ __forceinline__ void finalize_unit(const StepParams &sp, int32_t u, u
         }
         for (int i = total + 1 + lane; i < p.max_sel; i += 32) sel[i] = -1;
     }
-    // every team CTA has read the old length (each published its list after reading it)
+    // every team CTA read the old length at its start, before it wrote its list
     if (grow && lane == 0) sp.ap.seq_len[u] = L;
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release_gpu(sp.ready + 2 * u + 1, 1);
 }
 }  // namespace
 
@@ -187,7 +202,9 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     const int32_t C = p.pieces;
     const int32_t u = (int32_t)blockIdx.x / C, cidx = (int32_t)blockIdx.x % C;
     // (the append warp reads the length inside the append)
-    const int32_t L_prev = warp == kAppendWarp ? 0 : ld_volatile_s32(p.seq_len + u);
+    const int32_t L_prev = ld_volatile_s32(p.seq_len + u);
+    const int32_t launches = ld_volatile_s32(sp.epoch + u);
+    const uint32_t tag = launch_tag(launches);
     const bool grow = L_prev >= 0 && L_prev < p.max_ctx;
     const int32_t L = grow ? L_prev + 1 : L_prev;
     const int32_t nb_c = L > 0 ? (L - 1) / kBlock : 0;
@@ -196,9 +213,11 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     const int32_t s0 = cidx * ns / C, s1 = (cidx + 1) * ns / C;
     const int n_sc = s1 - s0;
     const int32_t b1 = min(s1 * kBPS, nb_c);
-    // and its piece [d_lo, d_hi) of the unit's max_sel decode slots (C <= max_sel: never empty)
-    const int32_t d_lo = cidx * p.max_sel / C, d_hi = (cidx + 1) * p.max_sel / C;
-    const int n_items = d_hi - d_lo;
+    // and its piece of the decode slots: [e_lo, e_hi) of the k_e + 1 slots of Gamma_e (slots < k_e)
+    // and the local block (slot k_e), then [q_lo, q_hi) of the k_q slots of Gamma_q \ Gamma_e
+    const int32_t e_lo = cidx * (p.k_e + 1) / C, e_hi = (cidx + 1) * (p.k_e + 1) / C;
+    const int32_t q_lo = cidx * p.k_q / C, q_hi = (cidx + 1) * p.k_q / C;
+    const int n_items = (e_hi - e_lo) + (q_hi - q_lo);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStepS; ++s) {
@@ -211,13 +230,86 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     }
     __syncthreads();
 
-    if (warp == kAppendWarp) {
+    if (warp == kSelectWarp) {
+        // ---------------- selection warp ----------------
         if (cidx == 0) {
             append_unit(sp.ap, u, lane, sp.ap.e_new[u], false);  // fences its writes
             __syncwarp();
-            if (lane == 0) st_release_gpu(sp.ready + 2 * u, 1);
+            if (lane == 0) st_release_gpu(sp.appended + u, 1);
         }
-        append_barrier_arrive();
+        // Gamma_e as this step's append left it, in a bitmap over the candidates, ready for the
+        // finalize while the lists are being scored (only the team's last CTA uses it)
+        int ok = 1;
+        if (lane == 0) {
+            ok = flag_wait(sp.appended + u);
+            if (!ok) set_error(p.err, NOSA_EFLAG_TIMEOUT);
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        __syncwarp();
+        const int32_t ne = L > 0 ? min(max(__ldcg(sp.gamma_n + u), 0), p.k_e) : 0;
+        int32_t ge_reg[kMaxKe / 32];
+#pragma unroll
+        for (int i = 0; i < kMaxKe / 32; ++i) {
+            const int j = lane + 32 * i;
+            ge_reg[i] = (j < ne) ? __ldcg(sp.gamma_e + (int64_t)u * p.k_e + j) : -1;
+        }
+        const int32_t nw = (nb_c + 31) >> 5;
+        for (int i = lane; i < nw; i += 32) bitmap[i] = 0;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kMaxKe / 32; ++i) {
+            const int32_t id = ge_reg[i];
+            if (id >= 0 && id < nb_c) atomicOr(&bitmap[id >> 5], 1u << (id & 31));
+        }
+        __syncwarp();
+        // the consumers' eight lists, merged; then published to the team
+        lists_wait();
+        uint64_t l8[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) l8[w] = lists[w * 32 + lane];
+        uint64_t list = merge_lists(l8, kConsWarps, lane);
+        if (cidx > 0) {
+            // to team CTA 0, tagged
+            st_relaxed_u64(sp.part_keys + ((int64_t)u * C + cidx) * 32 + lane, pack_key(list, tag));
+        } else {
+            // the other team CTAs' lists, eight at a time, each polled until it carries this tag
+            const uint64_t *all = sp.part_keys + (int64_t)u * C * 32;
+            bool ok_all = true;
+            for (int c0 = 1; c0 < C; c0 += 8) {
+                const int n = min(8, C - c0);
+                uint64_t w[8];
+                bool have[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    w[j] = 0ull;
+                    have[j] = j >= n;
+                }
+                const long long t0 = clock64();
+                while (true) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (!have[j]) {
+                            w[j] = ld_relaxed_u64(all + (int64_t)(c0 + j) * 32 + lane);
+                            have[j] = (uint32_t)(w[j] & kTagMask) == tag;
+                        }
+                    }
+                    bool mine = true;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) mine = mine && have[j];
+                    if (__all_sync(0xFFFFFFFFu, mine)) break;
+                    if (__shfl_sync(0xFFFFFFFFu, (int)(clock64() - t0 > kWaitCycles), 0)) {
+                        ok_all = false;
+                        break;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) l8[j] = (j < n && have[j]) ? unpack_key(w[j]) : 0ull;
+                list_merge(list, merge_lists(l8, n, lane), lane);
+            }
+            if (!ok_all && lane == 0) set_error(p.err, NOSA_EFLAG_TIMEOUT);
+            finalize_unit(sp, u, list, L, nb_c, grow, bitmap, tag, lane);
+        }
+        select_done_arrive();
         return;
     }
 
@@ -236,7 +328,9 @@ __global__ void __launch_bounds__(kStepThreads, 1)
             }
         }
         it = __shfl_sync(0xFFFFFFFFu, it, 0);
-        // decode slots [a, b): the block of each, fetched by the warp 32 at a time; lane 0 issues
+        // decode slots [a, b) (slot j < k_e: Gamma_e[j]; k_e: the local block; k_e + 1 + i: the
+        // i-th block of Gamma_q \ Gamma_e): the block of each, fetched by the warp 32 at a time;
+        // lane 0 issues
         auto issue = [&](int32_t a, int32_t b, int32_t ne) {
             for (int32_t xb = a; xb < b && !s_abort; xb += 32) {
                 const int nb = min(32, b - xb);
@@ -249,7 +343,21 @@ __global__ void __launch_bounds__(kStepThreads, 1)
                     } else if (j == p.k_e) {
                         lb = L > 0 ? nb_c : -1;
                     } else {
-                        lb = __ldcg(sp.rest + (int64_t)u * p.k_q + (j - p.k_e - 1));
+                        // written (tagged) by team CTA 0's selection warp: poll until current
+                        const uint32_t *slot = sp.rest + (int64_t)u * p.k_q + (j - p.k_e - 1);
+                        uint32_t w = ld_relaxed_u32(slot);
+                        const long long t0 = clock64();
+                        while ((w & kTagMask) != tag) {
+                            if (clock64() - t0 > kWaitCycles) {
+                                set_error(p.err, NOSA_EFLAG_TIMEOUT);
+                                s_abort = 1;
+                                w = tag;
+                                break;
+                            }
+                            __nanosleep(32);
+                            w = ld_relaxed_u32(slot);
+                        }
+                        lb = (int32_t)(w >> kTagBits) - 1;
                     }
                 }
                 for (int k = 0; k < nb; ++k, ++it) {
@@ -283,23 +391,15 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         // Gamma_e and the local block need the append (its new row, and Gamma_e as it left it)
         int ok = 1;
         if (lane == 0 && !s_abort) {
-            ok = flag_wait(sp.ready + 2 * u);
+            ok = flag_wait(sp.appended + u);
             if (ok) fence_proxy_async_global();  // the copies below read what the append wrote
             else { s_abort = 1; set_error(p.err, NOSA_EFLAG_TIMEOUT); }
         }
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (ok && !s_abort) {
             const int32_t ne = L > 0 ? min(max(__ldcg(sp.gamma_n + u), 0), p.k_e) : 0;
-            issue(d_lo, min(d_hi, p.k_e + 1), ne);
-            if (d_hi > p.k_e + 1 && !s_abort) {
-                // the Gamma_q slots need the selection
-                if (lane == 0) {
-                    ok = flag_wait(sp.ready + 2 * u + 1);
-                    if (!ok) { s_abort = 1; set_error(p.err, NOSA_EFLAG_TIMEOUT); }
-                }
-                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-                if (ok) issue(max(d_lo, p.k_e + 1), d_hi, ne);
-            }
+            issue(e_lo, e_hi, ne);
+            if (q_hi > q_lo && !s_abort) issue(p.k_e + 1 + q_lo, p.k_e + 1 + q_hi, ne);
         }
         // never leave with copies in flight
         if (lane == 0)
@@ -376,42 +476,8 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         const int32_t blk = (s0 + it) * kBPS + wq * (kRows / kSubPerBlock) + beta;
         list_offer(list, (offer && blk < b1) ? select_key(sc, blk) : 0ull, lane);
     }
-    tree_merge(list, lists, warp, lane);
-
-    // ---- publish; the team's last CTA forms Gamma_q and S(t) ----
-    append_barrier_sync();
-    bool fin = true;
-    if (C > 1) {
-        if (warp == 0) {
-            sp.part_keys[((int64_t)u * C + cidx) * 32 + lane] = list;
-            __syncwarp();
-            // counted with release semantics; the last CTA acquires the others' lists
-            if (lane == 0) s_last = ((int32_t)atom_add_acq_rel_gpu(sp.score_ctr + u, 1u) == C - 1);
-        }
-        consumer_sync();
-        fin = s_last;
-        if (fin) {
-            if (ctid == 0) sp.score_ctr[u] = 0;
-            const uint64_t *all = sp.part_keys + (int64_t)u * C * 32;
-            list = 0;  // a warp without lists contributes an empty one
-            for (int c0 = warp; c0 < C; c0 += 4 * kConsWarps) {
-                uint64_t k[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int cj = c0 + j * kConsWarps;
-                    k[j] = cj < C ? __ldcg(all + (int64_t)cj * 32 + lane) : 0ull;
-                }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {  // conditions uniform over the warp
-                    if (c0 + j * kConsWarps >= C) break;
-                    if (c0 == warp && j == 0) list = k[0];
-                    else list_merge(list, k[j], lane);
-                }
-            }
-            tree_merge(list, lists, warp, lane);
-        }
-    }
-    if (fin && warp == 0) finalize_unit(sp, u, list, L, nb_c, grow, bitmap, lane);
+    lists[warp * 32 + lane] = list;  // to the selection warp; the consumers go on
+    lists_arrive();
 
     // ---- attention over this CTA's piece of the decode list ----
     uint32_t qf[8][2];
@@ -437,6 +503,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         if (lane == 0) mbar_arrive(&empty[s]);
     }
     fold_groups(st, scratch, grp, wq, r, c, sig);
+    select_done_wait();  // the selection warp's flag and writes come before this CTA's count
     uint16_t *out = p.out + (int64_t)u * p.G * kD;
     float *part = p.part + (int64_t)blockIdx.x * kPartFloats;
     for (int idx = ctid; idx < p.G * kD; idx += kConsThreads) {
@@ -447,10 +514,10 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         else store_partial(part, h, d, M, acc, lsum);
     }
     if (C == 1) {
-        // this CTA is the whole team: its producer is past both flags
+        // this CTA is the whole team: its producer is past the flag and the Gamma_q slots
         if (ctid == 0) {
-            sp.ready[2 * u] = 0;
-            sp.ready[2 * u + 1] = 0;
+            sp.appended[u] = 0;
+            sp.epoch[u] = launches + 1;
         }
         return;
     }
@@ -459,15 +526,15 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     if (ctid == 0) s_last = ((int32_t)atom_add_acq_rel_gpu(p.counter + u, 1u) == C - 1);
     consumer_sync();
     if (!s_last) return;
-    // the unit's last piece: every team CTA has finished, so no one reads the flags any more
+    // the unit's last piece: every team CTA has finished, so no one reads the flag or the tags any more
     if (ctid == 0) {
         p.counter[u] = 0;
-        sp.ready[2 * u] = 0;
-        sp.ready[2 * u + 1] = 0;
+        sp.appended[u] = 0;
+        sp.epoch[u] = launches + 1;
     }
     const float *src0 = p.part + (int64_t)u * C * kPartFloats;
     if (C <= kOnePassPieces) {
-        merge_pieces_onepass(src0, kPartFloats, C, p.G, out, ctid);
+        merge_pieces_onepass<kOnePassPieces>(src0, kPartFloats, C, p.G, out, ctid);
     } else {
         const MergeScratch ms = merge_scratch(scratch, C);
         for (int t = ctid; t < C; t += kConsThreads) ms.src[t] = src0 + (int64_t)t * kPartFloats;

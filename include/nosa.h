@@ -301,7 +301,9 @@ int nosa_append_select(const nosa_config *cfg, const nosa_state *st, const uint1
  * Each unit is served by a team of CTAs that wait on one another (bounded
  * waits); with several CTAs per unit the kernel is launched cooperatively, so
  * the whole grid (at most one CTA per SM) must be able to run at once:
- * NOSA_ERR_CUDA if it cannot.  NOSA_ERR_UNSUPPORTED with offload == 1 (the
+ * NOSA_ERR_CUDA if it cannot.  The workspace keeps a count of launches per
+ * unit (it tags what the team's CTAs pass to one another), so after the
+ * one-time zero fill it must serve only this state's nosa_fused_step calls.  NOSA_ERR_UNSUPPORTED with offload == 1 (the
  * cache sync runs between the selection and the decode) or NOSA_FLAG_FILL
  * (Gamma_e is formed after Gamma_q there).
  */

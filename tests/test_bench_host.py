@@ -17,10 +17,15 @@ def _args(workload, **kw):
 
 
 def test_every_workload_uses_the_fused_launch_and_describes_itself():
+    # the device-store workloads run each layer's step in one launch, the offload workload the fused
+    # append + select (the cache sync runs between the selection and the decode there)
     for name, c in bench.WORKLOADS.items():
         assert c["fuse"] is True
+        assert c.get("step", False) is (not c["offload"])
         text = bench.describe(c, 2)
-        assert "append and select fused in one launch" in text and f"context {c['L']}" in text
+        want = "append and select fused in one launch" if c["offload"] else "(append, select, decode) in one launch"
+        assert want in text and f"context {c['L']}" in text
+    assert "append and select fused" in bench.describe(dict(bench.WORKLOADS["stack28-32k"], step=False), 2)
 
 
 def test_step_bytes_match_the_per_unit_formula():

@@ -93,22 +93,34 @@ def run_config(c, steps, seqs=None, seed=0, micro=1, dense_step=None, name=None,
     return st
 
 
-def test_mha_8k_full():
+# the device-store configurations run both ways: append + select, then decode (two launches), and
+# the fused step (one launch)
+PATHS = {"two launches": dict(step=False), "fused step": dict(step=True)}
+
+
+def _wl(name, path):
+    return dict(bench.WORKLOADS[name], **PATHS[path])
+
+
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_mha_8k_full(path):
     """1 layer, batch 1, 16/16 heads, 8K context, 32 steps: every unit, every step."""
-    run_config(dict(bench.WORKLOADS["mha-8k"]), steps=32, seqs=[0], name="mha-8k")
+    run_config(_wl("mha-8k", path), steps=32, seqs=[0], name=f"mha-8k {path}")
 
 
-def test_gqa_16k_full():
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_gqa_16k_full(path):
     """1 layer, batch 8, GQA 8:1, 16K context, 128 steps: every sequence and kv head, every step."""
-    run_config(dict(bench.WORKLOADS["gqa-16k"]), steps=128, seqs=list(range(8)), name="gqa-16k")
+    run_config(_wl("gqa-16k", path), steps=128, seqs=list(range(8)), name=f"gqa-16k {path}")
 
 
+@pytest.mark.parametrize("path", sorted(PATHS))
 @pytest.mark.parametrize("layer", [0, 27])
-def test_stack28_32k_layer(layer):
+def test_stack28_32k_layer(layer, path):
     """Batch 32, GQA 8:1, 32K context, layer 0 or 27 of the 28: all 64 decode steps, first and last
     sequence, both kv heads, plus the dense comparator at the last step."""
-    run_config(dict(bench.WORKLOADS["stack28-32k"]), steps=64, dense_step=63, layer=layer,
-               name=f"stack28-32k layer {layer}")
+    run_config(_wl("stack28-32k", path), steps=64, dense_step=63, layer=layer,
+               name=f"stack28-32k layer {layer} {path}")
 
 
 @pytest.mark.parametrize("layer", [0, 27])
@@ -129,6 +141,7 @@ def test_sweep_cell(B, L, k, offload):
     """The sweep (1 layer, 16 q / 2 kv heads, k_e = 0.75 k): every (context, k, device / pinned host)
     cell at batch 8, and every batch at 128K and k = 64, in the launch configuration the sweep times;
     4 decode steps on two sampled units, the first sequence's kv head 0 and the last one's kv head 1."""
-    c = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=k // 4, k_e=3 * k // 4, steps=64, offload=offload, fuse=True)
+    c = dict(layers=1, B=B, Hq=16, Hkv=2, L=L, k_q=k // 4, k_e=3 * k // 4, steps=64, offload=offload, fuse=True,
+             step=True)
     run_config(c, steps=4, micro=1, units=[(0, 0), (B - 1, 1)],
                name=f"sweep B={B} L={L} k={k} {'offload' if offload else 'device'}")

@@ -68,7 +68,7 @@ def test_unfused_stack28_32k_one_layer():
 
 @pytest.mark.parametrize("offload", [False, True])
 def test_layer_decode_step(offload):
-    """NosaLayer.decode_step, the one-call step the README shows (fused append + select, cache sync,
-    sparse decode)."""
+    """NosaLayer.decode_step, the one-call step the README shows (the device store: nosa_fused_step;
+    the offload store: fused append + select, cache sync, sparse decode)."""
     _run(H.Scenario(B=2, Hq=16, Hkv=2, k_q=4, k_e=12, L0=64 * 21 + 30, steps=70, offload=offload, seed=15,
                     layer_step=True))
