@@ -32,19 +32,23 @@ def _full_layer(fused):
     return cfg, lay
 
 
-@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("fused", [False, True, "step"])
 def test_append_past_capacity_sets_the_flag_and_keeps_the_state(fused):
+    # separate launches, append + select in one launch, and the whole step in one launch
     cfg, lay = _full_layer(fused)
     kn, vn = _rows(2, 3).view(2, 1, 128), _rows(2, 4).view(2, 1, 128)
     en = torch.zeros((2, 1), dtype=torch.float32, device="cuda")
     q = _rows(8, 5).view(1, 8, 128)
     out = torch.empty((1, 8, 128), dtype=torch.int16, device="cuda")
-    if fused:
+    if fused == "step":
+        lay.fused_step(kn, vn, en, q, out)
+    elif fused:
         lay.append_select(kn, vn, en, q)
     else:
         lay.append(kn, vn, en, 1)
         lay.select(q)
-    lay.sparse_decode(q, out)
+    if fused != "step":
+        lay.sparse_decode(q, out)
     torch.cuda.synchronize()
     assert lay.read_error(clear=False) & nosa.EFLAG_CAPACITY
     assert lay.seq_len.cpu().tolist() == [128, 128]  # nothing appended

@@ -99,3 +99,15 @@ def test_refusals():
         with pytest.raises(nosa.NosaError) as ei:
             lay.fused_step(kv, kv, e, q, torch.empty_like(q))
         assert ei.value.code == code
+    # a workspace below nosa_workspace_bytes: refused before any launch, the state untouched
+    cfg = nosa.make_config(2, 16, 2, 16, 48, 4096)
+    lay = nosa.NosaLayer(cfg)
+    q = torch.zeros((2, 16, 128), dtype=torch.int16, device="cuda")
+    kv = torch.zeros((4, 1, 128), dtype=torch.int16, device="cuda")
+    e = torch.zeros((4, 1), dtype=torch.float32, device="cuda")
+    small = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(nosa.NosaError) as ei:
+        nosa.nosa_fused_step(cfg, lay.state, kv, kv, e, q, lay.sel, lay.nsel, lay.gq, torch.empty_like(q), small)
+    assert ei.value.code == nosa.ERR_CAPACITY
+    torch.cuda.synchronize()
+    assert lay.seq_len.cpu().tolist() == [0, 0, 0, 0]
