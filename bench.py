@@ -371,6 +371,27 @@ def step_bytes(wl):
     return wl.L * wl.units * per_unit
 
 
+def algo_bytes(c, U, Bm, Lctx, nsel_mean):
+    """Algorithmic bytes per launch of each kernel, for one layer of one micro-batch of Bm sequences
+    (U units) at context Lctx, with nsel_mean blocks attended per unit (|S(t)|, the local block
+    included).  Select: the pooled keys of the (Lctx - 1) // 64 candidates and the G query heads of each
+    unit.  Decode: the K, V and eviction logits of the attended blocks, the queries and the outputs.
+    Append: the new K, V rows and logit.  The fused launches add up their parts."""
+    nb_c = (Lctx - 1) // 64
+    blk = 64 * D * 2 * 2 + 64 * 4  # one block: keys + values (bf16) + eviction logits (fp32)
+    a = {
+        "select": U * (nb_c * 4 * D * ck_elem(c) + (c["Hq"] // c["Hkv"]) * D * 2),
+        "decode": U * nsel_mean * blk + 2 * Bm * c["Hq"] * D * 2,
+        "append": U * (2 * D * 2 + 4),
+    }
+    a["append_select"] = a["select"] + a["append"]
+    a["step"] = a["append_select"] + a["decode"]
+    n_res = min(c["k_e"], nb_c) + 1  # Gamma_e + the local block
+    a["resident"] = U * n_res * blk + Bm * c["Hq"] * D * 2
+    a["rest"] = U * max(nsel_mean - n_res, 0) * blk + 2 * Bm * c["Hq"] * D * 2
+    return a
+
+
 def time_idempotent(wl, name, reps, flush=None):
     """Average device time of one launch of a kernel (select, decode, the split decode's resident /
     rest passes, the dense comparator, the fused append + select, or the fused step): a CUDA graph of
@@ -791,17 +812,7 @@ def run_nosa(args, c, rank, world, dev):
     nsel_mean = nsel_sum / max(nsel_n, 1)
     hbm_peak, peak_kind = load_peaks()
     U, Lctx = wl.units_m, c["L"] + step_i
-    nb_c = (Lctx - 1) // 64
-    algo = {  # algorithmic bytes per launch (one layer of one micro-batch)
-        "select": U * (nb_c * 4 * D * ck_elem(c) + (c["Hq"] // c["Hkv"]) * D * 2),
-        "decode": U * nsel_mean * (64 * D * 2 * 2 + 64 * 4) + 2 * wl.Bm * c["Hq"] * D * 2,
-        "append": U * (2 * D * 2 + 4),
-    }
-    algo["append_select"] = algo["select"] + algo["append"]
-    algo["step"] = algo["append_select"] + algo["decode"]
-    n_res = min(c["k_e"], nb_c) + 1  # Gamma_e + the local block
-    algo["resident"] = U * n_res * (64 * D * 2 * 2 + 64 * 4) + wl.Bm * c["Hq"] * D * 2
-    algo["rest"] = U * max(nsel_mean - n_res, 0) * (64 * D * 2 * 2 + 64 * 4) + 2 * wl.Bm * c["Hq"] * D * 2
+    algo = algo_bytes(c, U, wl.Bm, Lctx, nsel_mean)
     kern = {}
     for name, ts in kt.items():
         avg = sum(ts) / len(ts)

@@ -98,3 +98,19 @@ def test_reference_arm_prints_one_contract_line(monkeypatch, capsys):
     assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     assert line["cpu_baseline"]["host"]["logical_cores"] >= 1
+
+
+def test_algorithmic_bytes_per_launch():
+    # stack28-32k, one layer: 64 units at 32K + 9 tokens of context, 65 blocks attended per unit
+    c = dict(bench.WORKLOADS["stack28-32k"])
+    a = bench.algo_bytes(c, U=64, Bm=32, Lctx=32768 + 9, nsel_mean=65.0)
+    nb_c = (32768 + 9 - 1) // 64
+    assert a["select"] == 64 * (nb_c * 2048 + 8 * 256)  # fp32 pooled keys: 4 x 128 x 4 B per block
+    assert a["decode"] == 64 * 65 * (32768 + 256) + 2 * 32 * 16 * 256
+    assert a["append"] == 64 * 516
+    assert a["step"] == a["select"] + a["append"] + a["decode"]  # the fused step reads each once
+    assert abs(a["step"] / 1e6 - 204.9) < 0.1  # 67.2 MB of pooled keys + 137.6 MB of blocks, queries, outputs
+    # bf16 pooled keys halve the select stream; the split decode's passes add up to the one-pass decode
+    b = bench.algo_bytes(dict(c, ck_bf16=True), U=64, Bm=32, Lctx=32768 + 9, nsel_mean=65.0)
+    assert b["select"] - 64 * 8 * 256 == (a["select"] - 64 * 8 * 256) / 2
+    assert a["resident"] + a["rest"] == a["decode"] + 32 * 16 * 256
